@@ -1,0 +1,116 @@
+"""Seeded synthetic inputs for the attention forward pass.
+
+This module only draws random numbers; it holds none of the method's
+arithmetic.  The tests feed the same tensors to the CUDA path and to the CPU
+oracle, and ``bench.py`` times the CUDA path on them.
+
+Every tensor is drawn on the CPU with ``torch.Generator`` in float32 from
+N(0, 1), multiplied by its standard deviation, then rounded to bfloat16
+(round-to-nearest-even), in the order q, k, v.  Layout is [B, H, N, d],
+contiguous, d fastest.
+
+The workload shapes follow the pages' description of the problem: sequence
+lengths from 128 to 16k, head dim 64 and 128, full, causal and block-sparse
+attention.  "N(0,3)" for the long workload is read as standard deviation 3
+(it is meant to widen the score range so the running max is rescaled often;
+std 3 gives score std ~9 at scale 1/sqrt(d), variance 3 only ~3).
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+MASK_BLOCK = 128
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool = False
+    seed: int = 0
+    qk_std: float = 1.0
+    v_std: float = 1.0
+    sparse_p: float | None = None  # keep probability of off-diagonal blocks
+    mask_seed: int | None = None
+    note: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def describe(self) -> str:
+        parts = [f"B={self.B},H={self.H},N={self.N},d={self.d}"]
+        parts.append("causal" if self.causal else "full")
+        if self.sparse_p is not None:
+            parts.append(f"block-sparse 128x128 diag+p={self.sparse_p}")
+        if self.qk_std != 1.0:
+            parts.append(f"Q,K std {self.qk_std}")
+        return " ".join(parts)
+
+
+# The five workloads: tiny full, small (full and causal), mid causal,
+# long full with a wide score range, block-sparse.
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 1, 128, 64, seed=0),
+    "small": Workload("small", 4, 8, 1024, 64, seed=1),
+    "small_causal": Workload("small_causal", 4, 8, 1024, 64, causal=True, seed=1),
+    "mid_causal": Workload("mid_causal", 2, 16, 4096, 128, causal=True, seed=2),
+    "long_full": Workload("long_full", 1, 16, 16384, 128, seed=3, qk_std=3.0),
+    "sparse": Workload("sparse", 2, 16, 8192, 64, seed=4, sparse_p=0.25, mask_seed=4),
+}
+
+
+def make_qkv(B, H, N, d, seed, qk_std=1.0, v_std=1.0):
+    """q, k, v as contiguous CPU bfloat16 tensors [B, H, N, d]."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    shape = (B, H, N, d)
+    q = (torch.randn(shape, generator=g, dtype=torch.float32) * qk_std).to(torch.bfloat16)
+    k = (torch.randn(shape, generator=g, dtype=torch.float32) * qk_std).to(torch.bfloat16)
+    v = (torch.randn(shape, generator=g, dtype=torch.float32) * v_std).to(torch.bfloat16)
+    return q, k, v
+
+
+def make_block_mask(B, H, N, p, seed, block=MASK_BLOCK):
+    """uint8 [B, H, nb, nb] block mask, nb = ceil(N / block), 1 = keep.
+
+    One mask per head (diagonal blocks always kept, off-diagonal blocks kept
+    independently with probability p), the same for every batch index.
+    """
+    nb = (N + block - 1) // block
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    keep = torch.rand((H, nb, nb), generator=g) < p
+    keep |= torch.eye(nb, dtype=torch.bool).unsqueeze(0)
+    return keep.to(torch.uint8).unsqueeze(0).expand(B, H, nb, nb).contiguous()
+
+
+def make_inputs(w: Workload):
+    """(q, k, v, block_mask or None) on the CPU for a workload."""
+    q, k, v = make_qkv(w.B, w.H, w.N, w.d, w.seed, w.qk_std, w.v_std)
+    mask = None
+    if w.sparse_p is not None:
+        mask = make_block_mask(w.B, w.H, w.N, w.sparse_p, w.mask_seed)
+    return q, k, v, mask
+
+
+def useful_flops(B, H, N, d, causal=False, block_mask=None):
+    """FLOPs credited to one forward pass: 4*B*H*N^2*d, halved when causal,
+    times the kept-block fraction when a block mask is given."""
+    f = 4.0 * B * H * N * N * d
+    if causal:
+        f *= 0.5
+    if block_mask is not None:
+        f *= float(block_mask.to(torch.float64).mean())
+    return f
+
+
+def algorithmic_bytes(B, H, N, d):
+    """HBM bytes of one forward pass if every tensor moves once:
+    bf16 Q, K, V read and O written (8*N*d per head) plus fp32 lse (4*N)."""
+    return float(B * H * (8 * N * d + 4 * N))
