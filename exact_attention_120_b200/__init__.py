@@ -1,0 +1,145 @@
+"""B200 (sm_100a) fused exact-attention forward: Python binding of the C ABI.
+
+The binding only marshals arguments: every step of the forward pass runs in
+the CUDA kernel behind ``libfa_b200.so`` (see ``include/fa.h``).  PyTorch is
+used for device memory and streams.  There is no CPU fallback: if the
+library is missing or the device is not an sm_100 GPU the calls raise.
+
+Functions with the C names take raw device addresses:
+
+* ``fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask)``
+* ``fa_fwd_stream(..., stream)``
+* ``fa_device_status(stream)``, ``fa_status_string(status)``
+
+and ``attention_forward(q, k, v, ...)`` is the tensor-level convenience that
+allocates ``o`` and ``lse`` and launches on torch's current stream.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "FaError", "library_path", "load_library", "fa_fwd", "fa_fwd_stream", "fa_device_status",
+    "fa_status_string", "fa_launches_per_call", "attention_forward", "FA_OK",
+    "FA_ERR_INVALID_ARGUMENT", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT",
+    "MASK_BLOCK",
+]
+
+FA_OK = 0
+FA_ERR_INVALID_ARGUMENT = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_CUDA = 3
+FA_ERR_DEVICE_TIMEOUT = 4
+MASK_BLOCK = 128
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+# Exported symbols of the library, with their ctypes signatures.
+_SIGNATURES = {
+    "fa_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
+               + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
+    "fa_fwd_stream": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
+                      + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                              ctypes.c_void_p]),
+    "fa_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "fa_last_cuda_error": (ctypes.c_int, []),
+    "fa_launches_per_call": (ctypes.c_int, []),
+}
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        name = fa_status_string(status) if _LIB is not None else str(status)
+        extra = ""
+        if status == FA_ERR_CUDA and _LIB is not None:
+            extra = f" (cuda error {_LIB.fa_last_cuda_error()})"
+        super().__init__(f"{what}: {name}{extra}" if what else f"{name}{extra}")
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "libfa_b200.so")
+
+
+def load_library():
+    """Load ``libfa_b200.so`` (raises if it was not built)."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise FileNotFoundError(
+                f"{path} is missing: build it with `python -m exact_attention_120_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask) -> int:
+    """C ``fa_fwd`` on raw device addresses (ints); returns the status code."""
+    return load_library().fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask)
+
+
+def fa_fwd_stream(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, stream) -> int:
+    """C ``fa_fwd_stream`` on raw device addresses and a cudaStream_t (int)."""
+    return load_library().fa_fwd_stream(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask,
+                                        stream)
+
+
+def fa_device_status(stream=None) -> int:
+    return load_library().fa_device_status(stream)
+
+
+def fa_status_string(status: int) -> str:
+    return load_library().fa_status_string(status).decode()
+
+
+def fa_launches_per_call() -> int:
+    return load_library().fa_launches_per_call()
+
+
+def attention_forward(q, k, v, causal=False, block_mask=None, scale=None, out=None, lse=None,
+                      stream=None):
+    """O, lse = attention(q, k, v) through ``fa_fwd_stream``.
+
+    q, k, v: CUDA bfloat16 tensors [B, H, N, d], contiguous, d in {64, 128}.
+    block_mask: None or a CUDA uint8 tensor [B, H, ceil(N/128), ceil(N/128)].
+    scale: defaults to 1/sqrt(d).  Returns (o bf16 [B,H,N,d], lse fp32 [B,H,N]).
+    """
+    import torch
+
+    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must share one [B, H, N, d] shape")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA bfloat16 tensors")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    mask_ptr = None
+    if block_mask is not None:
+        nb = (N + MASK_BLOCK - 1) // MASK_BLOCK
+        if (block_mask.dtype != torch.uint8 or not block_mask.is_cuda
+                or tuple(block_mask.shape) != (B, H, nb, nb) or not block_mask.is_contiguous()):
+            raise ValueError(f"block_mask must be a contiguous CUDA uint8 [B,H,{nb},{nb}] tensor")
+        mask_ptr = block_mask.data_ptr()
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        st = fa_fwd_stream(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                           B, H, N, d, float(scale), int(bool(causal)), mask_ptr, stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_stream")
+    return out, lse

@@ -1,0 +1,217 @@
+// Host side of the C ABI declared in include/fa.h: argument validation,
+// TMA descriptor encoding, per-device set-up and the kernel launch.
+//
+// Nothing here computes any part of attention; every step of the forward
+// pass runs in fa_fwd_kernel.  There is no CPU fallback: without an sm_100
+// device the entry points return FA_ERR_UNSUPPORTED.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_fwd_kernel.cuh"
+
+namespace {
+
+// Device-side status word (FA_OK or FA_ERR_DEVICE_TIMEOUT), one per device.
+__device__ int g_fa_status = 0;
+
+thread_local int t_last_cuda_error = 0;
+
+constexpr unsigned long long kWaitTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s per wait
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceState {
+  std::once_flag once;
+  int status = FA_ERR_CUDA;  // result of the set-up
+  int num_sms = 0;
+  int* status_word = nullptr;  // device address of g_fa_status
+};
+
+DeviceState g_dev[kMaxDevices];
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_CUDA;
+}
+
+int setup_device(int dev, DeviceState& st) {
+  cudaDeviceProp prop;
+  cudaError_t e = cudaGetDeviceProperties(&prop, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (prop.major != 10 || prop.minor != 0) return FA_ERR_UNSUPPORTED;  // sm_100 only
+  st.num_sms = prop.multiProcessorCount;
+  e = cudaFuncSetAttribute(fa::fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           fa::Cfg<64>::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaFuncSetAttribute(fa::fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           fa::Cfg<128>::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e);
+  void* sym = nullptr;
+  e = cudaGetSymbolAddress(&sym, g_fa_status);
+  if (e != cudaSuccess) return cuda_fail(e);
+  st.status_word = static_cast<int*>(sym);
+  return FA_OK;
+}
+
+int get_device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  DeviceState& st = g_dev[dev];
+  std::call_once(st.once, [&] { st.status = setup_device(dev, st); });
+  if (st.status != FA_OK) return st.status;
+  *out = &st;
+  return FA_OK;
+}
+
+int get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode ? FA_OK : FA_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// True if the pointer is device (or managed) memory the GPU can address.
+bool is_device_pointer(const void* p) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error state of the query
+    return false;
+  }
+  return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+// [B*H][N][d] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle.
+int encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = static_cast<int>(r);
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                  int N, int d, float scale, int causal, const uint8_t* block_mask,
+                  void* cuda_stream) {
+  // ---- arguments (nothing is launched on error)
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARGUMENT;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARGUMENT;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARGUMENT;
+  const long long bh = (long long)B * H;
+  const long long nqt = (N + fa::kBM - 1) / fa::kBM;
+  const long long npairs = (nqt + 1) / 2;
+  if (bh > INT32_MAX || bh * npairs > INT32_MAX || (long long)N * d * 2 >= (1ll << 40))
+    return FA_ERR_UNSUPPORTED;  // 32-bit work indices and TMA stride limits
+  if (o == q || o == k || o == v) return FA_ERR_INVALID_ARGUMENT;
+
+  DeviceState* st = nullptr;
+  int rc = get_device_state(&st);
+  if (rc != FA_OK) return rc;
+  if (!is_device_pointer(q) || !is_device_pointer(k) || !is_device_pointer(v) ||
+      !is_device_pointer(o) || !is_device_pointer(lse) ||
+      (block_mask && !is_device_pointer(block_mask)))
+    return FA_ERR_INVALID_ARGUMENT;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+
+  // ---- parameters
+  fa::KernelParams p;
+  std::memset(&p, 0, sizeof(p));
+  if ((rc = encode_qkv_map(&p.tm_q, q, (int)bh, N, d)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_k, k, (int)bh, N, d)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_v, v, (int)bh, N, d)) != FA_OK) return rc;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.mask = block_mask;
+  p.N = N;
+  p.nqt = (int)nqt;
+  p.npairs = (int)npairs;
+  p.bh = (int)bh;
+  p.items = (int)(bh * npairs);
+  p.causal = causal;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.timeout_ns = kWaitTimeoutNs;
+  p.status = st->status_word;
+
+  // ---- launch: persistent grid, one CTA per SM
+  const int grid = p.items < st->num_sms ? p.items : st->num_sms;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (d == 64)
+    fa::fa_fwd_kernel<64><<<grid, fa::kThreads, fa::Cfg<64>::kSmemBytes, stream>>>(p);
+  else
+    fa::fa_fwd_kernel<128><<<grid, fa::kThreads, fa::Cfg<128>::kSmemBytes, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, float scale, int causal, const uint8_t* block_mask) {
+  return fa_fwd_stream(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, nullptr);
+}
+
+int fa_device_status(void* cuda_stream) {
+  DeviceState* st = nullptr;
+  int rc = get_device_state(&st);
+  if (rc != FA_OK) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  int value = 0;
+  cudaError_t e = cudaMemcpyAsync(&value, st->status_word, sizeof(int), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->status_word, 0, sizeof(int), stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return value == 0 ? FA_OK : value;
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARGUMENT: return "FA_ERR_INVALID_ARGUMENT";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_DEVICE_TIMEOUT: return "FA_ERR_DEVICE_TIMEOUT";
+    default: return "FA_UNKNOWN_STATUS";
+  }
+}
+
+int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+int fa_launches_per_call(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,529 @@
+// Fused exact-attention forward kernel for B200 (sm_100a).
+//
+// What it computes (per batch b, head h, query row i):
+//   O_i = sum_j softmax_j(scale * q_i . k_j) v_j over the visible keys j, and
+//   lse_i = ln sum_j exp(scale * q_i . k_j)
+// in one pass over the keys with the online softmax (AllenY's blog,
+// "FlashAttention" post, sections "从3-pass到2-pass" and "FlashAttention";
+// wmrh.cn FlashAttention article, "2.2 把 Online Softmax 嵌入注意力": one Q
+// block stays put while every K/V block streams past, with per-row running
+// max m, denominator l and an output accumulator corrected when m grows).
+// The N x N scores live only in tensor memory.
+//
+// Work unit: a pair of 128-row query tiles (2p, 2p+1) of one (b, h) -- the
+// Q-block-stationary split of "理解 Flash Attention" ("算法概述": one job per Q
+// block, streaming all of K and V), with two Q blocks sharing each K/V tile.
+// The grid is persistent: CTA c takes work units c, c + gridDim.x, ...
+//
+// Warp roles (320 threads, one CTA per SM, 512 tensor-memory columns):
+//   warps 0-3  softmax for query tile 2p   (thread t owns row t of the tile)
+//   warps 4-7  softmax for query tile 2p+1
+//   warp  8    MMA issue (one thread): S_q = Q_q K_j^T and O_q += P_q V_j
+//   warp  9    TMA producer: Q tiles, then K_j, V_j through a ring in smem
+//
+// Tensor memory (fp32 columns, lane = tile row):
+//   S_0 [0,128)  S_1 [128,256)  O_0 [256,256+D)  O_1 [384,384+D)
+//   P_q (bf16 pairs, 64 columns) overwrites the first half of S_q once the
+//   softmax has read S_q into registers; the PV MMA reads P_q from there.
+//
+// Online softmax in base 2: with c = scale * log2(e), each row keeps a
+// reference max m_ref (in units of c * score) and l = sum 2^(c s - m_ref).
+// The reference is moved (and O, l rescaled by 2^(m_old - m_new), the
+// concatenation rule of "理解 Flash Attention", "瓦片注意力计算") only when the
+// tile max exceeds it by more than kRescaleLog2 -- otherwise p <= 2^8, which
+// fp32 and bf16 hold without loss.  l sums the bf16-rounded p that the PV MMA
+// consumes, so O / l is an exact convex combination of V rows.
+//
+// Every wait on an mbarrier is bounded (globaltimer); on expiry the CTA
+// records FA_ERR_DEVICE_TIMEOUT, all roles leave their loops, in-flight TMA
+// loads and MMAs are drained and tensor memory is released before exit.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace fa {
+
+constexpr int kBM = 128;  // query rows per tile (= MMA M)
+constexpr int kBN = 128;  // keys per tile (= mask block)
+constexpr int kThreads = 320;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kStatusTimeout = 4;  // == FA_ERR_DEVICE_TIMEOUT
+
+struct KernelParams {
+  CUtensorMap tm_q;  // 3-D maps over [B*H][N][D] bf16, box 64 x 128 x 1, 128B swizzle
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  __nv_bfloat16* o;
+  float* lse;
+  const uint8_t* mask;  // nullptr or [B*H][nqt][nqt]
+  int N;
+  int nqt;     // query (= key) tiles per head
+  int npairs;  // work units per head
+  int bh;      // B * H
+  int items;   // bh * npairs
+  int causal;
+  float scale_log2;  // scale * log2(e)
+  unsigned long long timeout_ns;
+  int* status;  // device status word
+};
+
+template <int D>
+struct Cfg {
+  static_assert(D == 64 || D == 128, "head dim 64 or 128");
+  static constexpr int kBoxes = D / 64;          // 64-column TMA boxes per tile
+  static constexpr int kBoxBytes = 128 * 128;    // 128 rows x 128 B
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
+  // q_full, q_empty, full[S], empty[S], s_full[2], p_full[2], o_full[2], o_empty[2], mma_done
+  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 384;
+};
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, A K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+  return (1u << 4)                           // D format: f32
+         | (1u << 7)                         // A format: bf16
+         | (1u << 10)                        // B format: bf16
+         | ((b_mn_major ? 1u : 0u) << 16)    // B major-ness
+         | ((uint32_t)(N >> 3) << 17)        // N / 8
+         | ((uint32_t)(M >> 4) << 24);       // M / 16
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
+// lbo/sbo in bytes.  K-major tiles: sbo = 1024 (8 rows x 128 B), lbo unused.
+// MN-major tiles: lbo = distance between 64-element column blocks, sbo = 1024.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void decode_item(const KernelParams& p, int w, int& bh, int& pair) {
+  if (p.causal) {  // longest rows first, all heads interleaved
+    pair = p.npairs - 1 - w / p.bh;
+    bh = w % p.bh;
+  } else {  // all pairs of one head together: that head's K/V stays in L2
+    bh = w / p.npairs;
+    pair = w % p.npairs;
+  }
+}
+
+// Bit l set <=> key tile j0 + l is visible to query tile qt (whole warp calls).
+__device__ __forceinline__ uint32_t keep_bits(const KernelParams& p, int bh, int qt, int j0,
+                                              int lane) {
+  const int j = j0 + lane;
+  bool k = (qt < p.nqt) && (j < p.nqt);
+  if (k && p.causal) k = (j <= qt);
+  if (k && p.mask != nullptr) k = p.mask[((size_t)bh * p.nqt + qt) * p.nqt + j] != 0;
+  return __ballot_sync(0xffffffffu, k);
+}
+
+// Bounded wait for the phase of `bar` with parity `parity`.  Returns false if
+// this wait timed out or, when `honor_abort`, the CTA is aborting because
+// another role timed out.  Drain waits pass honor_abort = false: they must see
+// their copies land (or time out) even while aborting.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                      const KernelParams& p, bool honor_abort = true) {
+  if (ptx::mbar_test(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_test(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (honor_abort && *abort_flag) return false;
+      if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+        *abort_flag = 1;
+        atomicCAS(p.status, 0, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ KernelParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+
+  const uint32_t sQ = base + C::kOffQ;
+  const uint32_t sRing = base + C::kOffRing;
+  const uint32_t bar0 = base + C::kOffBar;
+  const uint32_t bQFull = bar0, bQEmpty = bar0 + 8;
+  auto bFull = [&](int s) { return bar0 + 16 + 8u * s; };
+  auto bEmpty = [&](int s) { return bar0 + 16 + 8u * (C::kStages + s); };
+  const uint32_t bq = bar0 + 16 + 16u * C::kStages;
+  auto bSFull = [&](int q) { return bq + 8u * q; };
+  auto bPFull = [&](int q) { return bq + 16 + 8u * q; };
+  auto bOFull = [&](int q) { return bq + 32 + 8u * q; };
+  auto bOEmpty = [&](int q) { return bq + 48 + 8u * q; };
+  const uint32_t bMmaDone = bq + 64;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bQFull, 1);
+    ptx::mbar_init(bQEmpty, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      ptx::mbar_init(bFull(s), 1);
+      ptx::mbar_init(bEmpty(s), 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      ptx::mbar_init(bSFull(q), 1);
+      ptx::mbar_init(bPFull(q), 128);
+      ptx::mbar_init(bOFull(q), 1);
+      ptx::mbar_init(bOEmpty(q), 128);
+    }
+    ptx::mbar_init(bMmaDone, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async_smem();
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    ptx::prefetch_tensormap(&p.tm_q);
+    ptx::prefetch_tensormap(&p.tm_k);
+    ptx::prefetch_tensormap(&p.tm_v);
+  }
+  if (warp == kMmaWarp) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------ TMA producer ---
+    uint32_t it = 0;       // K/V ring loads issued
+    uint32_t nq = 0;       // Q loads issued
+    bool ok = true;
+    for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
+      int bh, pair;
+      decode_item(p, w, bh, pair);
+      const int qt0 = 2 * pair, qt1 = qt0 + 1;
+      const int nvalid = (qt1 < p.nqt) ? 2 : 1;
+      if (lane == 0) {
+        ok = wait_bar(bQEmpty, (nq & 1u) ^ 1u, abort_flag, p);
+        if (ok) {
+          ptx::mbar_arrive_expect_tx(bQFull, nvalid * C::kTileBytes);
+          for (int q = 0; q < nvalid; ++q)
+            for (int bx = 0; bx < C::kBoxes; ++bx)
+              ptx::tma_load_3d(sQ + q * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q, bQFull, bx * 64,
+                               (qt0 + q) * kBM, bh);
+        }
+      }
+      ++nq;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      const int jend = p.causal ? min(p.nqt, qt0 + nvalid) : p.nqt;
+      for (int j0 = 0; j0 < jend && ok; j0 += 32) {
+        uint32_t u = keep_bits(p, bh, qt0, j0, lane) | keep_bits(p, bh, qt1, j0, lane);
+        while (u != 0 && ok) {
+          const int j = j0 + __ffs(u) - 1;
+          u &= u - 1;
+          if (lane == 0) {
+            for (int t = 0; t < 2 && ok; ++t) {  // K_j then V_j
+              const int slot = it % C::kStages;
+              ok = wait_bar(bEmpty(slot), ((it / C::kStages) & 1u) ^ 1u, abort_flag, p);
+              if (ok) {
+                ptx::mbar_arrive_expect_tx(bFull(slot), C::kTileBytes);
+                const CUtensorMap* map = t == 0 ? &p.tm_k : &p.tm_v;
+                for (int bx = 0; bx < C::kBoxes; ++bx)
+                  ptx::tma_load_3d(sRing + slot * C::kTileBytes + bx * C::kBoxBytes, map,
+                                   bFull(slot), bx * 64, j * kBN, bh);
+                ++it;
+              }
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+      }
+    }
+    // Drain: every load issued must have landed before the CTA may exit.
+    if (lane == 0) {
+      const uint32_t first = it > (uint32_t)C::kStages ? it - C::kStages : 0u;
+      for (uint32_t r = first; r < it; ++r)
+        wait_bar(bFull(r % C::kStages), (r / C::kStages) & 1u, abort_flag, p, false);
+      if (nq > 0) wait_bar(bQFull, (nq - 1) & 1u, abort_flag, p, false);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------- MMA issuer ---
+    constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
+    constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
+    uint32_t it = 0;              // ring slots consumed (mirrors the producer)
+    uint32_t nq = 0;              // Q tiles consumed
+    uint32_t pwait[2] = {0, 0};   // p_full phases consumed
+    uint32_t nitems[2] = {0, 0};  // work units seen per query slot
+    int64_t v_ready = -1;         // ring index of the newest V whose load was awaited
+    bool ok = true;
+    for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
+      int bh, pair;
+      decode_item(p, w, bh, pair);
+      const int qt0 = 2 * pair, qt1 = qt0 + 1;
+      const bool valid1 = qt1 < p.nqt;
+      int64_t pend[2] = {-1, -1};  // ring index of the V owed a PV MMA, per query slot
+      bool need_oe[2] = {nitems[0] > 0, valid1 && nitems[1] > 0};
+      uint32_t npv[2] = {0, 0};
+      int64_t prev_v = -1;
+
+      // O_q += P_q V  for the pending V of slot q.
+      auto issue_pv = [&](int q) -> bool {
+        if (!wait_bar(bPFull(q), pwait[q] & 1u, abort_flag, p)) return false;
+        ++pwait[q];
+        ptx::tc_fence_after();
+        const int64_t vr = pend[q];
+        if (vr > v_ready) {
+          if (!wait_bar(bFull((int)(vr % C::kStages)), (uint32_t)(vr / C::kStages) & 1u, abort_flag, p))
+            return false;
+          v_ready = vr;
+          ptx::tc_fence_after();
+        }
+        if (need_oe[q]) {  // the previous unit's epilogue has read O_q
+          if (!wait_bar(bOEmpty(q), (nitems[q] - 1) & 1u, abort_flag, p)) return false;
+          need_oe[q] = false;
+          ptx::tc_fence_after();
+        }
+        const uint32_t vbase = sRing + (uint32_t)(vr % C::kStages) * C::kTileBytes;
+        const uint32_t tO = tmem + (q ? C::kTmemO1 : C::kTmemO0);
+        const uint32_t tP = tmem + (q ? C::kTmemS1 : C::kTmemS0);
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, C::kBoxBytes, 1024);
+          ptx::mma_ts(tO, tP + kk * 8, bdesc, kIdescPV, (npv[q] > 0 || kk > 0) ? 1u : 0u);
+        }
+        ++npv[q];
+        pend[q] = -1;
+        return true;
+      };
+
+      if (lane == 0) {
+        ok = wait_bar(bQFull, nq & 1u, abort_flag, p);
+        ptx::tc_fence_after();
+      }
+      ++nq;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      const int jend = p.causal ? min(p.nqt, qt0 + (valid1 ? 2 : 1)) : p.nqt;
+      for (int j0 = 0; j0 < jend && ok; j0 += 32) {
+        const uint32_t k0 = keep_bits(p, bh, qt0, j0, lane);
+        const uint32_t k1 = keep_bits(p, bh, qt1, j0, lane);
+        uint32_t u = k0 | k1;
+        while (u != 0 && ok) {
+          const int l = __ffs(u) - 1;
+          u &= u - 1;
+          if (lane == 0) {
+            const uint32_t kr = it, vr = it + 1;
+            it += 2;
+            const int kslot = kr % C::kStages;
+            ok = wait_bar(bFull(kslot), (kr / C::kStages) & 1u, abort_flag, p);
+            ptx::tc_fence_after();
+            const bool keep[2] = {((k0 >> l) & 1u) != 0, ((k1 >> l) & 1u) != 0};
+            for (int q = 0; q < 2 && ok; ++q) {
+              if (!keep[q]) continue;
+              if (pend[q] >= 0) ok = issue_pv(q);
+              if (!ok) break;
+              // S_q = Q_q K_j^T
+              const uint32_t qbase = sQ + q * C::kTileBytes;
+              const uint32_t kbase = sRing + kslot * C::kTileBytes;
+              const uint32_t tS = tmem + (q ? C::kTmemS1 : C::kTmemS0);
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+                ptx::mma_ss(tS, smem_desc_sw128(qbase + off, 16, 1024),
+                            smem_desc_sw128(kbase + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+              }
+              ptx::mma_commit(bSFull(q));
+              pend[q] = vr;
+            }
+            if (ok) ptx::mma_commit(bEmpty(kslot));  // K_j no longer needed
+            for (int q = 0; q < 2 && ok; ++q)
+              if (!keep[q] && pend[q] >= 0) ok = issue_pv(q);
+            if (ok && prev_v >= 0) ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
+            prev_v = vr;
+          }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+      }
+      if (lane == 0 && ok) {
+        // Every S MMA of this unit is issued: Q may be replaced once they finish.
+        ptx::mma_commit(bQEmpty);
+        for (int q = 0; q < 2 && ok; ++q)
+          if (pend[q] >= 0) ok = issue_pv(q);
+        if (ok && prev_v >= 0) ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
+        if (ok) {
+          if (npv[0] > 0) ptx::mma_commit(bOFull(0));
+          if (valid1 && npv[1] > 0) ptx::mma_commit(bOFull(1));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ++nitems[0];
+      if (valid1) ++nitems[1];
+    }
+    // Drain: every MMA issued must be complete before tensor memory is freed.
+    if (lane == 0) {
+      ptx::mma_commit(bMmaDone);
+      wait_bar(bMmaDone, 0, abort_flag, p, false);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- softmax ---
+    const int q = warp >> 2;               // query slot 0 or 1
+    const int row_in_tile = threadIdx.x & 127;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (q ? C::kTmemS1 : C::kTmemS0);
+    const uint32_t tO = tmem + lane_base + (q ? C::kTmemO1 : C::kTmemO0);
+    const float sl = p.scale_log2;
+    uint32_t swait = 0, owait = 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
+      int bh, pair;
+      decode_item(p, w, bh, pair);
+      const int qt = 2 * pair + q;
+      if (qt >= p.nqt) continue;
+      const int row = qt * kBM + row_in_tile;
+      float m_ref = -INFINITY;  // reference max, in units of c * score
+      float l = 0.f;            // sum of bf16-rounded 2^(c s - m_ref)
+      int n = 0;                // tiles processed
+      const int jend = p.causal ? min(p.nqt, qt + 1) : p.nqt;
+      for (int j0 = 0; j0 < jend && ok; j0 += 32) {
+        uint32_t kb = keep_bits(p, bh, qt, j0, lane);
+        while (kb != 0 && ok) {
+          const int j = j0 + __ffs(kb) - 1;
+          kb &= kb - 1;
+          ok = wait_bar(bSFull(q), swait & 1u, abort_flag, p);
+          ok = __all_sync(0xffffffffu, ok);
+          ++swait;
+          if (!ok) break;
+          ptx::tc_fence_after();
+          uint32_t r[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, r[c]);
+          ptx::tmem_wait_ld();
+          float s[128];
+#pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c >> 5][c & 31]);
+          // Mask: causal diagonal tile and the ragged tail of the sequence.
+          int lim = 127;
+          if (p.causal && j == qt) lim = row_in_tile;
+          const int tail = p.N - j * kBN - 1;
+          if (tail < lim) lim = tail;
+          if (lim < 127) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c > lim) s[c] = -INFINITY;
+          }
+          float mx[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx[t] = s[t];
+#pragma unroll
+          for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
+          float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          const float m_new = fmaxf(m_ref, tmax * sl);
+          // Move the reference max only when the new one exceeds it by more than
+          // 2^kRescaleLog2 (always on the first visible tile: m_ref = -inf).
+          const bool rescale = m_new > m_ref + kRescaleLog2;
+          float alpha = 1.f;
+          if (rescale) {
+            alpha = ptx::ex2(m_ref - m_new);  // 0 when m_ref = -inf
+            l *= alpha;
+            m_ref = m_new;
+          }
+          const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+          uint32_t pk[2][32];
+          float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float a = ptx::ex2(fmaf(s[2 * c], sl, -m_use));
+            const float b = ptx::ex2(fmaf(s[2 * c + 1], sl, -m_use));
+            const uint32_t w2 = ptx::pack_bf16x2(a, b);
+            pk[c >> 5][c & 31] = w2;
+            ls[c & 3] += __uint_as_float(w2 << 16) + __uint_as_float(w2 & 0xFFFF0000u);
+          }
+          l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+          ptx::tmem_st32(tS, pk[0]);
+          ptx::tmem_st32(tS + 32, pk[1]);
+          // O holds earlier tiles: rescale it in place.  tcgen05.ld/st are
+          // warp-collective, so the warp rescales together (alpha = 1 for rows
+          // whose reference did not move).
+          if (n > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t t[32];
+              ptx::tmem_ld32(tO + 32 * c, t);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
+              ptx::tmem_st32(tO + 32 * c, t);
+            }
+          }
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bPFull(q));
+          ++n;
+        }
+      }
+      if (!ok) break;
+      // ------------------------------------------------------- epilogue ---
+      if (n > 0) {
+        ok = wait_bar(bOFull(q), owait & 1u, abort_flag, p);
+        ok = __all_sync(0xffffffffu, ok);
+        ++owait;
+        if (!ok) break;
+        ptx::tc_fence_after();
+      }
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const bool in_range = row < p.N;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)bh * p.N + (in_range ? row : 0)) * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t t[32];
+        if (n > 0) {
+          ptx::tmem_ld32(tO + 32 * c, t);
+          ptx::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) t[e] = 0u;
+        }
+        uint32_t pkd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pkd[e] = ptx::pack_bf16x2(__uint_as_float(t[2 * e]) * inv, __uint_as_float(t[2 * e + 1]) * inv);
+        if (in_range) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            orow[c * 4 + v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bOEmpty(q));
+      if (in_range)
+        p.lse[(size_t)bh * p.N + row] =
+            (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,108 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) fused exact-attention forward pass.
+ *
+ * The operation
+ * -------------
+ * For every batch index b and head h, with query rows i and key rows j of
+ * one sequence of length N and head dimension d:
+ *
+ *     S_ij  = scale * sum_t Q[b,h,i,t] * K[b,h,j,t]
+ *     O_i   = sum_{j in vis(i)} softmax_j(S_i.) * V[b,h,j,:]
+ *     lse_i = ln sum_{j in vis(i)} exp(S_ij)
+ *
+ * This is scaled dot-product attention as stated in "理解 Flash Attention：在
+ * Triton 中从头编写算法" (section "什么是注意力"), computed exactly (wmrh.cn
+ * FlashAttention article, introduction: no accuracy is traded for speed) in
+ * one pass with the online softmax of AllenY's blog "FlashAttention" post
+ * (sections "从3-pass到2-pass" and "FlashAttention"): the N x N score matrix is
+ * never written to memory.  lse is the natural-log logsumexp of the scaled
+ * scores of each row (kept so a backward pass can recompute S).
+ *
+ * Visibility vis(i): every key; intersected with {j <= i} when `causal` is 1;
+ * intersected with {j : block_mask[b,h,i/128,j/128] != 0} when `block_mask`
+ * is non-NULL (block-sparse attention: a masked 128 x 128 block contributes
+ * nothing and is never loaded or multiplied).  A row whose vis(i) is empty
+ * gets O_i = 0 and lse_i = -inf.
+ *
+ * Layouts and types (all buffers are owned by the caller; the library
+ * allocates nothing per call and keeps no pointer after the call returns):
+ *   q, k, v, o   device memory, bfloat16, contiguous [B, H, N, d] (d fastest),
+ *                16-byte aligned.  o may not alias q, k or v.
+ *   lse          device memory, float32, contiguous [B, H, N], 4-byte aligned.
+ *   block_mask   NULL, or device memory, uint8, contiguous
+ *                [B, H, ceil(N/128), ceil(N/128)], 1 (non-zero) = keep.
+ *   d            64 or 128.
+ *   scale        finite and > 0 (usually 1/sqrt(d)).
+ *   causal       0 or 1.
+ *   N            any value >= 1; a ragged last tile is masked inside the kernel.
+ *
+ * Errors: every entry point returns an fa_status.  Argument errors are found
+ * before anything is launched.  Launches are asynchronous: a fault inside the
+ * kernel surfaces at the caller's next synchronisation; a device-side wait
+ * that exceeded its time limit is reported by fa_device_status().  No C++
+ * exception crosses this interface.  The entry points may be called from
+ * several host threads; per-device set-up is done once, under a lock.
+ */
+#ifndef FA_B200_FA_H_
+#define FA_B200_FA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FA_MASK_BLOCK 128
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+typedef enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARGUMENT = 1, /* null/misaligned/host pointer, bad size, scale, causal */
+  FA_ERR_UNSUPPORTED = 2,      /* d not in {64,128}, not an sm_100 device, size limits */
+  FA_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed: see fa_last_cuda_error() */
+  FA_ERR_DEVICE_TIMEOUT = 4    /* a device-side wait gave up (reported by fa_device_status) */
+} fa_status;
+
+/*
+ * Fused attention forward on the legacy default stream (stream 0).
+ * Writes o [B,H,N,d] and lse [B,H,N]; see the header comment for meaning.
+ */
+FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, float scale, int causal, const uint8_t* block_mask);
+
+/*
+ * The same, enqueued on `cuda_stream` (a cudaStream_t; NULL = legacy default
+ * stream).  The call returns once the kernel is enqueued.
+ */
+FA_API int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                  int N, int d, float scale, int causal, const uint8_t* block_mask,
+                  void* cuda_stream);
+
+/*
+ * Reads and clears the device-side status word of the current device after
+ * synchronising `cuda_stream`.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT (a
+ * kernel's wait on one of its own barriers exceeded the time limit; the
+ * kernel then stopped early and released its resources, and its outputs
+ * are undefined) or FA_ERR_CUDA.
+ */
+FA_API int fa_device_status(void* cuda_stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+FA_API const char* fa_status_string(int status);
+
+/* The cudaError_t value behind the last FA_ERR_CUDA on this host thread. */
+FA_API int fa_last_cuda_error(void);
+
+/* Number of kernel launches one fa_fwd call makes (constant: 1). */
+FA_API int fa_launches_per_call(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_FA_H_ */

@@ -1,0 +1,69 @@
+"""The C-ABI library builds, loads and exports every function include/fa.h
+declares; argument checks that precede any CUDA call work without a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_120_b200 import build as build_mod
+import exact_attention_120_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return fa.load_library()
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names.update(re.findall(r"^\s*(?:FA_API\s+)?(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert {"fa_fwd", "fa_fwd_stream", "fa_device_status", "fa_status_string"} <= names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID_ARGUMENT"), (2, "FA_ERR_UNSUPPORTED"),
+                       (3, "FA_ERR_CUDA"), (4, "FA_ERR_DEVICE_TIMEOUT")]:
+        assert fa.fa_status_string(code) == name
+    assert fa.fa_status_string(99) == "FA_UNKNOWN_STATUS"
+    assert fa.fa_launches_per_call() == 1
+
+
+def test_argument_errors_before_any_cuda_call(lib):
+    p = 1 << 20  # never dereferenced: every case fails validation first
+    base = [p, p, p, p * 2, p * 3, 1, 1, 128, 64, 0.125, 0, None]
+
+    def call(**kw):
+        a = list(base)
+        names = ["q", "k", "v", "o", "lse", "B", "H", "N", "d", "scale", "causal", "mask"]
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return fa.fa_fwd(*a)
+
+    assert call(q=None) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(lse=None) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(B=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(N=-5) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(scale=float("inf")) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(scale=0.0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(causal=3) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(d=256) == fa.FA_ERR_UNSUPPORTED
+    assert call(q=p + 8) == fa.FA_ERR_INVALID_ARGUMENT  # not 16-byte aligned
+    assert call(o=p) == fa.FA_ERR_INVALID_ARGUMENT      # o aliases q
+    assert call(B=1 << 16, H=1 << 16) == fa.FA_ERR_UNSUPPORTED  # B*H beyond 32 bits
