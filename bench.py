@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one fa_fwd launch over one batch of the workload (default: the
+long full-attention workload B=1, H=16, N=16384, d=128, Q/K std 3 -- the
+d=128, N>=4096 full-attention case the throughput target is stated on).
+Inputs are seeded and synthetic, resident in HBM when the timed region starts,
+and larger than L2 (Q, K, V, O = 256 MB per step), so no L2 flush is needed.
+
+Rank 0 prints ONE JSON line.  ``value`` is the whole-job TFLOP/s (useful
+FLOPs 4*B*H*N^2*d, halved when causal, times the kept-block fraction when
+block-sparse), timed with CUDA events on the launching stream, max over
+ranks.  ``e2e`` times the same metric through the public API with pinned host
+buffers, copies included.  ``roofline`` relates the kernel to the measured
+dense-bf16 tensor peak.  ``cpu_baseline`` times the float64 CPU oracle on a
+bounded sample of the same workload.  ``--impl reference`` times that oracle
+alone as the reference arm.
+
+Multi-GPU (launched by torchrun): ranks share nothing on the data path; each
+rank runs the full workload shape on its own batch slice (weak scaling).
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_attention_120_b200 import sharding  # noqa: E402
+from exact_attention_120_b200.workloads import (WORKLOADS, algorithmic_bytes, make_inputs,  # noqa: E402
+                                                useful_flops)
+
+METRIC = "fused attention fwd TFLOP/s (bf16, causal & full) and % of dense BF16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAK_TFLOPS = 1590.0
+KERNEL_SOURCES = ("exact_attention_120_b200/csrc/fa_fwd_kernel.cuh",
+                  "exact_attention_120_b200/csrc/ptx.cuh",
+                  "exact_attention_120_b200/csrc/fa_api.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+THROTTLE_BITS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), \
+            "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_PEAK_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, only if it was
+    taken on the current kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = rec.get(workload)
+    if not entry or entry.get("kernel_hash") != kernel_hash():
+        return None
+    return float(entry["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    def __init__(self, torch_device, period_s=0.02):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            props = __import__("torch").cuda.get_device_properties(torch_device)
+            bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id,
+                                        props.pci_device_id)
+            try:
+                self._handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except pynvml.NVMLError:
+                self._handle = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: clocks reported as unknown
+            self._handle = None
+
+    def _run(self):
+        nv = self._nvml
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self._handle))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        names = sorted(n for bit, n in THROTTLE_BITS.items() if self.reasons & bit and n != "gpu_idle")
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(w, q, k, v, mask, rows_per_chunk, budget_s=None, max_chunks=None, start=0):
+    """Time the float64 oracle on successive chunks of query rows of the
+    workload (head-major order), until `budget_s` seconds or `max_chunks`.
+    Returns (useful_flops, seconds, rows)."""
+    import numpy as np
+
+    import oracle
+
+    total_rows = w.B * w.H * w.N
+    flops = 0.0
+    rows_done = 0
+    t_total = 0.0
+    chunk = 0
+    while True:
+        r0 = (start + chunk * rows_per_chunk) % total_rows
+        idx = [(r0 + i) % total_rows for i in range(rows_per_chunk)]
+        sample = [(i // (w.H * w.N), (i // w.N) % w.H, i % w.N) for i in idx]
+        t0 = time.perf_counter()
+        oracle.attention_ref_rows(q, k, v, w.scale, sample, causal=w.causal,
+                                  block_mask=None if mask is None else mask)
+        t_total += time.perf_counter() - t0
+        for (b, h, i) in sample:
+            vis = oracle.visible_mask(w.N, w.N, w.causal,
+                                      None if mask is None else mask[b, h], rows=np.array([i]))
+            flops += 4.0 * w.d * float(vis.sum())
+        rows_done += len(sample)
+        chunk += 1
+        if (budget_s is not None and t_total >= budget_s) or (max_chunks is not None and chunk >= max_chunks):
+            break
+    return flops, t_total, rows_done
+
+
+def numpy_inputs(q, k, v, mask):
+    import torch
+
+    f = lambda t: t.to(torch.float64).numpy()  # noqa: E731  exact bf16 -> fp64
+    return f(q), f(k), f(v), (None if mask is None else mask.numpy())
+
+
+def run_reference(args, info):
+    """Reference arm: the float64 CPU oracle as it stands, on host cores."""
+    if not info.is_root:
+        return 0
+    w = WORKLOADS[args.workload]
+    q, k, v, mask = make_inputs(w)
+    qn, kn, vn, mn = numpy_inputs(q, k, v, mask)
+    rows = args.reference_rows
+    cores = blas_threads()
+    oracle_sample(w, qn, kn, vn, mn, rows, max_chunks=max(1, args.warmup))  # warm-up
+    step_s, step_f = [], []
+    for s in range(args.steps):
+        f, t, _ = oracle_sample(w, qn, kn, vn, mn, rows, max_chunks=1, start=(s + 1) * rows * 7)
+        step_f.append(f)
+        step_s.append(t)
+    value = sum(step_f) / sum(step_s) / 1e12
+    sample = (f"{rows} query rows per step (complete rows of S over all N={w.N} keys), "
+              f"head-major order; float64 NumPy/BLAS oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world_size,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(step_s) / len(step_s),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, info.world_size),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, world):
+    return {"workload": f"{w.name}: {w.describe()}, scale 1/sqrt(d), seed {w.seed}",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "block_sparse": w.sparse_p is not None, "global_batch": w.B * world, "seq_len": w.N,
+            "parallelism": "replicas" if world == 1 else f"dp{world} (independent batch slices)",
+            "l2": "inputs larger than L2 (Q, K, V, O = %d MB per step); no flush"
+                  % (algorithmic_bytes(w.B, w.H, w.N, w.d) // 2**20)}
+
+
+def run_ours(args, info):
+    import torch
+
+    import exact_attention_120_b200 as fa
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device (the kernel has no CPU path)")
+    dev = torch.device("cuda", info.local_rank)
+    torch.cuda.set_device(dev)
+    sharding.init_process_group(info, "nccl")
+    fa.load_library()
+
+    w = WORKLOADS[args.workload]
+    wr = dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank))
+    q, k, v, mask = make_inputs(wr)
+    flops = useful_flops(w.B, w.H, w.N, w.d, w.causal, mask)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    md = None if mask is None else mask.to(dev)
+    od = torch.empty_like(qd)
+    ld = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ptrs = (qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), ld.data_ptr())
+    mptr = None if md is None else md.data_ptr()
+
+    def launch():
+        st = fa.fa_fwd_stream(*ptrs, w.B, w.H, w.N, w.d, w.scale, int(w.causal), mptr,
+                              stream.cuda_stream)
+        if st != fa.FA_OK:
+            raise fa.FaError(st, "fa_fwd_stream")
+
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize(dev)
+    st = fa.fa_device_status(stream.cuda_stream)
+    if st != fa.FA_OK:
+        raise fa.FaError(st, "device status after warm-up")
+
+    # ---- device-timed region: K launches, inputs resident in HBM
+    sampler = ClockSampler(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sharding.barrier(dev)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        launch()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    sharding.barrier(dev)
+    ms = e0.elapsed_time(e1)
+    ms_max = sharding.max_over_ranks(ms, dev)
+    ms_step = ms_max / args.steps
+    st = fa.fa_device_status(stream.cuda_stream)
+    if st != fa.FA_OK:
+        raise fa.FaError(st, "device status after timed region")
+
+    # ---- end to end: pinned host inputs -> device -> fa_fwd -> host outputs
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    hm = None if mask is None else mask.pin_memory()
+    ho = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    hl = torch.empty(ld.shape, dtype=ld.dtype).pin_memory()
+
+    def e2e_step():
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        if hm is not None:
+            md.copy_(hm, non_blocking=True)
+        fa.attention_forward(qd, kd, vd, causal=w.causal, block_mask=md, scale=w.scale, out=od,
+                             lse=ld)
+        ho.copy_(od, non_blocking=True)
+        hl.copy_(ld, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(min(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    sharding.barrier(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sharding.max_over_ranks(e0.elapsed_time(e1), dev) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (0 if hm is None else hm.numel())
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    clocks = sampler.summary()
+    if info.world_size > 1:
+        import torch.distributed as dist
+
+        allc = [None] * info.world_size
+        dist.all_gather_object(allc, clocks)
+        clocks = dict(clocks)
+        clocks["reasons"] = sorted({r for c in allc for r in c["reasons"]})
+    sharding.destroy()
+    if not info.is_root:
+        return 0
+
+    peak, peak_sus, peak_src = load_peaks()
+    achieved = flops / (ms_step * 1e-3) / 1e12  # one launch per step
+    value = info.world_size * achieved
+    cpu = None
+    if info.world_size == 1 and not args.no_cpu_baseline:
+        qn, kn, vn, mn = numpy_inputs(q, k, v, mask)
+        f, t, rows = oracle_sample(w, qn, kn, vn, mn, args.cpu_rows, budget_s=args.cpu_budget)
+        cpu = {"value": f / t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{rows} query rows of {w.name} (complete rows over all N={w.N} keys, "
+                         f"head-major from row 0), {t:.1f} s of float64 NumPy/BLAS oracle"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world_size,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) draws, bf16)", "config": workload_config(w, info.world_size),
+        "pct_of_dense_bf16_peak": 100.0 * achieved / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": load_traffic(w.name),
+                     "peak_kind": f"{peak_src} burst dense bf16",
+                     "frac_of_sustained_peak": achieved / peak_sus,
+                     "algorithmic_bytes": algorithmic_bytes(w.B, w.H, w.N, w.d),
+                     "flops_per_launch": flops},
+        "e2e": {"value": info.world_size * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * fa.fa_launches_per_call(),
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "kernel_hash": kernel_hash(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="long_full", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per timed chunk")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--reference-rows", type=int, default=256, help="oracle rows per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    info = sharding.rank_info_from_env()
+    if info.world_size != args.gpus:
+        if info.world_size == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 must be launched with torchrun (one process per GPU)")
+    if args.impl == "reference":
+        return run_reference(args, info)
+    return run_ours(args, info)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
