@@ -15,11 +15,14 @@
 // block, streaming all of K and V), with two Q blocks sharing each K/V tile.
 // The grid is persistent: CTA c takes work units c, c + gridDim.x, ...
 //
-// Warp roles (320 threads, one CTA per SM, 512 tensor-memory columns):
-//   warps 0-3  softmax for query tile 2p   (thread t owns row t of the tile)
-//   warps 4-7  softmax for query tile 2p+1
-//   warp  8    MMA issue (one thread): S_q = Q_q K_j^T and O_q += P_q V_j
-//   warp  9    TMA producer: Q tiles, then K_j, V_j through a ring in smem
+// Warp roles (384 threads, one CTA per SM, 512 tensor-memory columns):
+//   warp  0    MMA issue (one thread): S_q = Q_q K_j^T and O_q += P_q V_j
+//   warp  1    TMA producer: Q tiles, then K_j, V_j through a ring in smem
+//   warps 2-3  idle
+//   warps 4-7  softmax for query tile 2p   (thread t owns row t of the tile)
+//   warps 8-11 softmax for query tile 2p+1
+// The issuing warps have the lowest ids: warp schedulers favour them over the
+// long-running softmax warps that share their SM sub-partitions.
 //
 // Tensor memory (fp32 columns, lane = tile row):
 //   S_0 [0,128)  S_1 [128,256)  O_0 [256,256+D)  O_1 [384,384+D)
@@ -49,9 +52,10 @@ namespace fa {
 
 constexpr int kBM = 128;  // query rows per tile (= MMA M)
 constexpr int kBN = 128;  // keys per tile (= mask block)
-constexpr int kThreads = 320;
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
+constexpr int kThreads = 384;
+constexpr int kMmaWarp = 0;
+constexpr int kLoadWarp = 1;
+constexpr int kFirstSoftmaxWarp = 4;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStatusTimeout = 4;  // == FA_ERR_DEVICE_TIMEOUT
@@ -150,6 +154,105 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// Whole-warp bounded wait: every lane polls, the result is warp-uniform.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          const KernelParams& p) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag, p));
+}
+
+// Barrier addresses shared by the kernel and the MMA helpers.  Layout from
+// bar0: q_full, q_empty, full[S], empty[S], s_full[2], p_full[2], o_full[2],
+// o_empty[2], mma_done.
+template <int D> __device__ __forceinline__ uint32_t bar_full(uint32_t bar0, int s) { return bar0 + 16 + 8u * s; }
+template <int D> __device__ __forceinline__ uint32_t bar_q(uint32_t bar0) { return bar0 + 16 + 16u * Cfg<D>::kStages; }
+template <int D> __device__ __forceinline__ uint32_t bar_s_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 8u * q; }
+template <int D> __device__ __forceinline__ uint32_t bar_p_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 16 + 8u * q; }
+template <int D> __device__ __forceinline__ uint32_t bar_o_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 32 + 8u * q; }
+template <int D> __device__ __forceinline__ uint32_t bar_o_empty(uint32_t bar0, int q) { return bar_q<D>(bar0) + 48 + 8u * q; }
+
+// MMA-issuer state of one query slot.
+struct MmaSlot {
+  int64_t pend = -1;     // ring index of the V tile owed a PV MMA, or -1
+  uint32_t npv = 0;      // PV MMAs issued in this work unit
+  uint32_t pwait = 0;    // p_full phases consumed
+  uint32_t nitems = 0;   // work units seen with this slot valid
+  bool need_oe = false;  // must wait for the previous unit's epilogue first
+  __device__ __forceinline__ void begin_unit(bool valid) {
+    pend = -1;
+    npv = 0;
+    need_oe = valid && nitems > 0;
+  }
+  __device__ __forceinline__ void end_unit(bool valid) {
+    if (valid) ++nitems;
+  }
+};
+
+template <int D>
+struct MmaCtx {
+  uint32_t tmem, sQ, sRing;
+  volatile int* abort_flag;
+};
+
+// O_q += P_q V for the pending V of slot Q.  Called by the whole MMA warp
+// (warp-uniform); one elected lane issues.
+template <int D, int Q>
+__device__ __forceinline__ bool mma_issue_pv(const MmaCtx<D>& c, const KernelParams& p, MmaSlot& s,
+                                             int64_t& v_ready, uint32_t bar0) {
+  using C = Cfg<D>;
+  constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
+  if (!wait_warp(bar_p_full<D>(bar0, Q), s.pwait & 1u, c.abort_flag, p)) return false;
+  ++s.pwait;
+  ptx::tc_fence_after();
+  const int64_t vr = s.pend;
+  if (vr > v_ready) {
+    if (!wait_warp(bar_full<D>(bar0, (int)(vr % C::kStages)), (uint32_t)(vr / C::kStages) & 1u,
+                   c.abort_flag, p))
+      return false;
+    v_ready = vr;
+    ptx::tc_fence_after();
+  }
+  if (s.need_oe) {  // the previous unit's epilogue has read O_q
+    if (!wait_warp(bar_o_empty<D>(bar0, Q), (s.nitems - 1) & 1u, c.abort_flag, p)) return false;
+    s.need_oe = false;
+    ptx::tc_fence_after();
+  }
+  const uint32_t vbase = c.sRing + (uint32_t)(vr % C::kStages) * C::kTileBytes;
+  const uint32_t tO = c.tmem + (Q ? C::kTmemO1 : C::kTmemO0);
+  const uint32_t tP = c.tmem + (Q ? C::kTmemS1 : C::kTmemS0);
+  const uint32_t acc0 = s.npv > 0 ? 1u : 0u;
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk)
+    if (ptx::elect_one())
+      ptx::mma_ts(tO, tP + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::kBoxBytes, 1024), kIdescPV,
+                  kk > 0 ? 1u : acc0);
+  ++s.npv;
+  s.pend = -1;
+  return true;
+}
+
+// One kept K tile for slot Q: settle its pending PV, then S_q = Q_q K_j^T.
+// Warp-uniform, like mma_issue_pv.
+template <int D, int Q>
+__device__ __forceinline__ bool mma_slot_step(const MmaCtx<D>& c, const KernelParams& p, MmaSlot& s,
+                                              int64_t& v_ready, int kslot, uint32_t vr, uint32_t bar0) {
+  using C = Cfg<D>;
+  constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
+  if (s.pend >= 0 && !mma_issue_pv<D, Q>(c, p, s, v_ready, bar0)) return false;
+  const uint32_t qbase = c.sQ + Q * C::kTileBytes;
+  const uint32_t kbase = c.sRing + kslot * C::kTileBytes;
+  const uint32_t tS = c.tmem + (Q ? C::kTmemS1 : C::kTmemS0);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+    if (ptx::elect_one())
+      ptx::mma_ss(tS, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                  kIdescQK, kk > 0 ? 1u : 0u);
+  }
+  if (ptx::elect_one()) ptx::mma_commit(bar_s_full<D>(bar0, Q));
+  s.pend = vr;
+  return true;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ KernelParams p) {
   using C = Cfg<D>;
@@ -162,14 +265,13 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   const uint32_t sRing = base + C::kOffRing;
   const uint32_t bar0 = base + C::kOffBar;
   const uint32_t bQFull = bar0, bQEmpty = bar0 + 8;
-  auto bFull = [&](int s) { return bar0 + 16 + 8u * s; };
+  auto bFull = [&](int s) { return bar_full<D>(bar0, s); };
   auto bEmpty = [&](int s) { return bar0 + 16 + 8u * (C::kStages + s); };
-  const uint32_t bq = bar0 + 16 + 16u * C::kStages;
-  auto bSFull = [&](int q) { return bq + 8u * q; };
-  auto bPFull = [&](int q) { return bq + 16 + 8u * q; };
-  auto bOFull = [&](int q) { return bq + 32 + 8u * q; };
-  auto bOEmpty = [&](int q) { return bq + 48 + 8u * q; };
-  const uint32_t bMmaDone = bq + 64;
+  auto bSFull = [&](int q) { return bar_s_full<D>(bar0, q); };
+  auto bPFull = [&](int q) { return bar_p_full<D>(bar0, q); };
+  auto bOFull = [&](int q) { return bar_o_full<D>(bar0, q); };
+  auto bOEmpty = [&](int q) { return bar_o_empty<D>(bar0, q); };
+  const uint32_t bMmaDone = bar_q<D>(bar0) + 64;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kOffMisc + 4);
 
@@ -218,106 +320,64 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       decode_item(p, w, bh, pair);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
       const int nvalid = (qt1 < p.nqt) ? 2 : 1;
-      if (lane == 0) {
-        ok = wait_bar(bQEmpty, (nq & 1u) ^ 1u, abort_flag, p);
-        if (ok) {
-          ptx::mbar_arrive_expect_tx(bQFull, nvalid * C::kTileBytes);
-          for (int q = 0; q < nvalid; ++q)
-            for (int bx = 0; bx < C::kBoxes; ++bx)
-              ptx::tma_load_3d(sQ + q * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q, bQFull, bx * 64,
-                               (qt0 + q) * kBM, bh);
-        }
+      ok = wait_warp(bQEmpty, (nq & 1u) ^ 1u, abort_flag, p);
+      if (ok && ptx::elect_one()) {
+        ptx::mbar_arrive_expect_tx(bQFull, nvalid * C::kTileBytes);
+        for (int q = 0; q < nvalid; ++q)
+          for (int bx = 0; bx < C::kBoxes; ++bx)
+            ptx::tma_load_3d(sQ + q * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q, bQFull, bx * 64,
+                             (qt0 + q) * kBM, bh);
       }
       ++nq;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       const int jend = p.causal ? min(p.nqt, qt0 + nvalid) : p.nqt;
       for (int j0 = 0; j0 < jend && ok; j0 += 32) {
         uint32_t u = keep_bits(p, bh, qt0, j0, lane) | keep_bits(p, bh, qt1, j0, lane);
         while (u != 0 && ok) {
           const int j = j0 + __ffs(u) - 1;
           u &= u - 1;
-          if (lane == 0) {
-            for (int t = 0; t < 2 && ok; ++t) {  // K_j then V_j
-              const int slot = it % C::kStages;
-              ok = wait_bar(bEmpty(slot), ((it / C::kStages) & 1u) ^ 1u, abort_flag, p);
-              if (ok) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {  // K_j then V_j
+            const int slot = it % C::kStages;
+            ok = ok && wait_warp(bEmpty(slot), ((it / C::kStages) & 1u) ^ 1u, abort_flag, p);
+            if (ok) {
+              if (ptx::elect_one()) {
                 ptx::mbar_arrive_expect_tx(bFull(slot), C::kTileBytes);
                 const CUtensorMap* map = t == 0 ? &p.tm_k : &p.tm_v;
                 for (int bx = 0; bx < C::kBoxes; ++bx)
                   ptx::tma_load_3d(sRing + slot * C::kTileBytes + bx * C::kBoxBytes, map,
                                    bFull(slot), bx * 64, j * kBN, bh);
-                ++it;
               }
+              ++it;
             }
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
         }
       }
     }
     // Drain: every load issued must have landed before the CTA may exit.
-    if (lane == 0) {
-      const uint32_t first = it > (uint32_t)C::kStages ? it - C::kStages : 0u;
-      for (uint32_t r = first; r < it; ++r)
-        wait_bar(bFull(r % C::kStages), (r / C::kStages) & 1u, abort_flag, p, false);
-      if (nq > 0) wait_bar(bQFull, (nq - 1) & 1u, abort_flag, p, false);
-    }
+    const uint32_t first = it > (uint32_t)C::kStages ? it - C::kStages : 0u;
+    for (uint32_t r = first; r < it; ++r)
+      wait_bar(bFull(r % C::kStages), (r / C::kStages) & 1u, abort_flag, p, false);
+    if (nq > 0) wait_bar(bQFull, (nq - 1) & 1u, abort_flag, p, false);
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issuer ---
-    constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
-    constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
+    MmaSlot slot0, slot1;         // per query slot state, kept in registers
     uint32_t it = 0;              // ring slots consumed (mirrors the producer)
     uint32_t nq = 0;              // Q tiles consumed
-    uint32_t pwait[2] = {0, 0};   // p_full phases consumed
-    uint32_t nitems[2] = {0, 0};  // work units seen per query slot
     int64_t v_ready = -1;         // ring index of the newest V whose load was awaited
     bool ok = true;
+    const MmaCtx<D> ctx{tmem, sQ, sRing, abort_flag};
     for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
       int bh, pair;
       decode_item(p, w, bh, pair);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
       const bool valid1 = qt1 < p.nqt;
-      int64_t pend[2] = {-1, -1};  // ring index of the V owed a PV MMA, per query slot
-      bool need_oe[2] = {nitems[0] > 0, valid1 && nitems[1] > 0};
-      uint32_t npv[2] = {0, 0};
+      slot0.begin_unit(true);
+      slot1.begin_unit(valid1);
       int64_t prev_v = -1;
-
-      // O_q += P_q V  for the pending V of slot q.
-      auto issue_pv = [&](int q) -> bool {
-        if (!wait_bar(bPFull(q), pwait[q] & 1u, abort_flag, p)) return false;
-        ++pwait[q];
-        ptx::tc_fence_after();
-        const int64_t vr = pend[q];
-        if (vr > v_ready) {
-          if (!wait_bar(bFull((int)(vr % C::kStages)), (uint32_t)(vr / C::kStages) & 1u, abort_flag, p))
-            return false;
-          v_ready = vr;
-          ptx::tc_fence_after();
-        }
-        if (need_oe[q]) {  // the previous unit's epilogue has read O_q
-          if (!wait_bar(bOEmpty(q), (nitems[q] - 1) & 1u, abort_flag, p)) return false;
-          need_oe[q] = false;
-          ptx::tc_fence_after();
-        }
-        const uint32_t vbase = sRing + (uint32_t)(vr % C::kStages) * C::kTileBytes;
-        const uint32_t tO = tmem + (q ? C::kTmemO1 : C::kTmemO0);
-        const uint32_t tP = tmem + (q ? C::kTmemS1 : C::kTmemS0);
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, C::kBoxBytes, 1024);
-          ptx::mma_ts(tO, tP + kk * 8, bdesc, kIdescPV, (npv[q] > 0 || kk > 0) ? 1u : 0u);
-        }
-        ++npv[q];
-        pend[q] = -1;
-        return true;
-      };
-
-      if (lane == 0) {
-        ok = wait_bar(bQFull, nq & 1u, abort_flag, p);
-        ptx::tc_fence_after();
-      }
+      ok = wait_warp(bQFull, nq & 1u, abort_flag, p);
+      ptx::tc_fence_after();
       ++nq;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
       const int jend = p.causal ? min(p.nqt, qt0 + (valid1 ? 2 : 1)) : p.nqt;
       for (int j0 = 0; j0 < jend && ok; j0 += 32) {
         const uint32_t k0 = keep_bits(p, bh, qt0, j0, lane);
@@ -326,63 +386,49 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         while (u != 0 && ok) {
           const int l = __ffs(u) - 1;
           u &= u - 1;
-          if (lane == 0) {
-            const uint32_t kr = it, vr = it + 1;
-            it += 2;
-            const int kslot = kr % C::kStages;
-            ok = wait_bar(bFull(kslot), (kr / C::kStages) & 1u, abort_flag, p);
-            ptx::tc_fence_after();
-            const bool keep[2] = {((k0 >> l) & 1u) != 0, ((k1 >> l) & 1u) != 0};
-            for (int q = 0; q < 2 && ok; ++q) {
-              if (!keep[q]) continue;
-              if (pend[q] >= 0) ok = issue_pv(q);
-              if (!ok) break;
-              // S_q = Q_q K_j^T
-              const uint32_t qbase = sQ + q * C::kTileBytes;
-              const uint32_t kbase = sRing + kslot * C::kTileBytes;
-              const uint32_t tS = tmem + (q ? C::kTmemS1 : C::kTmemS0);
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-                ptx::mma_ss(tS, smem_desc_sw128(qbase + off, 16, 1024),
-                            smem_desc_sw128(kbase + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-              }
-              ptx::mma_commit(bSFull(q));
-              pend[q] = vr;
-            }
-            if (ok) ptx::mma_commit(bEmpty(kslot));  // K_j no longer needed
-            for (int q = 0; q < 2 && ok; ++q)
-              if (!keep[q] && pend[q] >= 0) ok = issue_pv(q);
-            if (ok && prev_v >= 0) ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
-            prev_v = vr;
-          }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          const uint32_t kr = it, vr = it + 1;
+          it += 2;
+          const int kslot = kr % C::kStages;
+          ok = wait_warp(bFull(kslot), (kr / C::kStages) & 1u, abort_flag, p);
+          ptx::tc_fence_after();
+          const bool keep0 = ((k0 >> l) & 1u) != 0, keep1 = ((k1 >> l) & 1u) != 0;
+          // Slot q: pending O_q += P_q V first (P_q shares columns with S_q),
+          // then S_q = Q_q K_j^T.
+          if (ok && keep0) ok = mma_slot_step<D, 0>(ctx, p, slot0, v_ready, kslot, vr, bar0);
+          if (ok && keep1) ok = mma_slot_step<D, 1>(ctx, p, slot1, v_ready, kslot, vr, bar0);
+          if (ok && ptx::elect_one()) ptx::mma_commit(bEmpty(kslot));  // K_j no longer needed
+          // A slot that skips K_j still owes a PV on the previous V: issue it
+          // now so that V can be released.
+          if (ok && !keep0 && slot0.pend >= 0) ok = mma_issue_pv<D, 0>(ctx, p, slot0, v_ready, bar0);
+          if (ok && !keep1 && slot1.pend >= 0) ok = mma_issue_pv<D, 1>(ctx, p, slot1, v_ready, bar0);
+          if (ok && prev_v >= 0 && ptx::elect_one())
+            ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
+          prev_v = vr;
         }
       }
-      if (lane == 0 && ok) {
+      if (ok) {
         // Every S MMA of this unit is issued: Q may be replaced once they finish.
-        ptx::mma_commit(bQEmpty);
-        for (int q = 0; q < 2 && ok; ++q)
-          if (pend[q] >= 0) ok = issue_pv(q);
-        if (ok && prev_v >= 0) ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
-        if (ok) {
-          if (npv[0] > 0) ptx::mma_commit(bOFull(0));
-          if (valid1 && npv[1] > 0) ptx::mma_commit(bOFull(1));
+        if (ptx::elect_one()) ptx::mma_commit(bQEmpty);
+        if (slot0.pend >= 0) ok = mma_issue_pv<D, 0>(ctx, p, slot0, v_ready, bar0);
+        if (ok && slot1.pend >= 0) ok = mma_issue_pv<D, 1>(ctx, p, slot1, v_ready, bar0);
+        if (ok && prev_v >= 0 && ptx::elect_one())
+          ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
+        if (ok && ptx::elect_one()) {
+          if (slot0.npv > 0) ptx::mma_commit(bar_o_full<D>(bar0, 0));
+          if (valid1 && slot1.npv > 0) ptx::mma_commit(bar_o_full<D>(bar0, 1));
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      ++nitems[0];
-      if (valid1) ++nitems[1];
+      slot0.end_unit(true);
+      slot1.end_unit(valid1);
     }
     // Drain: every MMA issued must be complete before tensor memory is freed.
-    if (lane == 0) {
-      ptx::mma_commit(bMmaDone);
-      wait_bar(bMmaDone, 0, abort_flag, p, false);
-    }
+    if (ptx::elect_one()) ptx::mma_commit(bMmaDone);
     __syncwarp();
-  } else {
+    wait_bar(bMmaDone, 0, abort_flag, p, false);
+    __syncwarp();
+  } else if (warp >= kFirstSoftmaxWarp) {
     // ---------------------------------------------------------- softmax ---
-    const int q = warp >> 2;               // query slot 0 or 1
+    const int q = (warp - kFirstSoftmaxWarp) >> 2;  // query slot 0 or 1
     const int row_in_tile = threadIdx.x & 127;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + (q ? C::kTmemS1 : C::kTmemS0);
@@ -405,8 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         while (kb != 0 && ok) {
           const int j = j0 + __ffs(kb) - 1;
           kb &= kb - 1;
-          ok = wait_bar(bSFull(q), swait & 1u, abort_flag, p);
-          ok = __all_sync(0xffffffffu, ok);
+          ok = wait_warp(bSFull(q), swait & 1u, abort_flag, p);
           ++swait;
           if (!ok) break;
           ptx::tc_fence_after();
@@ -427,13 +472,15 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             for (int c = 0; c < 128; ++c)
               if (c > lim) s[c] = -INFINITY;
           }
-          float mx[8];
+          float mx[4];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) mx[t] = s[t];
+          for (int t = 0; t < 4; ++t) mx[t] = s[t];
 #pragma unroll
-          for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-          float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          for (int c = 4; c < 128; c += 8) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mx[t] = ptx::max3(mx[t], s[c + 2 * t], s[c + 2 * t + 1]);
+          }
+          const float tmax = ptx::max3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
           const float m_new = fmaxf(m_ref, tmax * sl);
           // Move the reference max only when the new one exceeds it by more than
           // 2^kRescaleLog2 (always on the first visible tile: m_ref = -inf).
@@ -444,16 +491,16 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             l *= alpha;
             m_ref = m_new;
           }
-          const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+          const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
           uint32_t pk[2][32];
           float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            const float a = ptx::ex2(fmaf(s[2 * c], sl, -m_use));
-            const float b = ptx::ex2(fmaf(s[2 * c + 1], sl, -m_use));
-            const uint32_t w2 = ptx::pack_bf16x2(a, b);
+            float x0, x1;
+            ptx::fma2(x0, x1, s[2 * c], s[2 * c + 1], sl, sl, neg_m, neg_m);
+            const uint32_t w2 = ptx::pack_bf16x2(ptx::ex2(x0), ptx::ex2(x1));
             pk[c >> 5][c & 31] = w2;
-            ls[c & 3] += __uint_as_float(w2 << 16) + __uint_as_float(w2 & 0xFFFF0000u);
+            ptx::add_bf16x2(ls[2 * (c & 1)], ls[2 * (c & 1) + 1], w2);
           }
           l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
           ptx::tmem_st32(tS, pk[0]);
@@ -481,8 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       if (!ok) break;
       // ------------------------------------------------------- epilogue ---
       if (n > 0) {
-        ok = wait_bar(bOFull(q), owait & 1u, abort_flag, p);
-        ok = __all_sync(0xffffffffu, ok);
+        ok = wait_warp(bOFull(q), owait & 1u, abort_flag, p);
         ++owait;
         if (!ok) break;
         ptx::tc_fence_after();
