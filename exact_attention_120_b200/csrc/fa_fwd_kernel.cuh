@@ -95,6 +95,38 @@ struct Cfg {
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 384;
 };
 
+// 2^x on the FMA pipe for two lanes (relieves the MUFU exp2 unit, which at
+// head dim 128 would otherwise run exactly as fast as the tensor cores eat
+// scores).  Cody-Waite range reduction x = n + f, n = round(x) via the
+// 1.5 * 2^23 rounding constant, f in [-1/2, 1/2]; 2^f from a degree-3
+// polynomial fitted for minimum relative error (max 7.6e-5, well under the
+// bf16 rounding that follows; the fit is exact_attention_120_b200/exp2_poly_fit.py);
+// 2^n added to the exponent field.  Arguments below -125 (masked scores are
+// -inf) give 2^-125.  Arguments never exceed +8 here (see kRescaleLog2).
+constexpr float kExp2Clamp = -125.0f;
+constexpr float kExp2Round = 12582912.0f;  // 1.5 * 2^23
+constexpr float kExp2C0 = 9.999282360e-01f;
+constexpr float kExp2C1 = 6.932609677e-01f;
+constexpr float kExp2C2 = 2.426085174e-01f;
+constexpr float kExp2C3 = 5.517049879e-02f;
+
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  x0 = fmaxf(x0, kExp2Clamp);
+  x1 = fmaxf(x1, kExp2Clamp);
+  float t0, t1, r0, r1, f0, f1, q0, q1;
+  ptx::add2(t0, t1, x0, x1, kExp2Round, kExp2Round);    // n in the low mantissa bits
+  ptx::add2(r0, r1, t0, t1, -kExp2Round, -kExp2Round);  // n as a float
+  ptx::fma2(f0, f1, r0, r1, -1.f, -1.f, x0, x1);        // f = x - n
+  ptx::fma2(q0, q1, f0, f1, kExp2C3, kExp2C3, kExp2C2, kExp2C2);
+  ptx::fma2(q0, q1, q0, q1, f0, f1, kExp2C1, kExp2C1);
+  ptx::fma2(q0, q1, q0, q1, f0, f1, kExp2C0, kExp2C0);
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// One pair in kPolyEvery of each row's exp2 goes through exp2_poly2.
+constexpr int kPolyEvery = 4;
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, A K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
   return (1u << 4)                           // D format: f32
@@ -472,11 +504,13 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             for (int c = 0; c < 128; ++c)
               if (c > lim) s[c] = -INFINITY;
           }
+          // Row max over the 128 scores: 4 chains of three-input max,
+          // s[0..7] seed the chains, s[8..127] are folded in pairs.
           float mx[4];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) mx[t] = s[t];
+          for (int t = 0; t < 4; ++t) mx[t] = fmaxf(s[2 * t], s[2 * t + 1]);
 #pragma unroll
-          for (int c = 4; c < 128; c += 8) {
+          for (int c = 8; c < 128; c += 8) {
 #pragma unroll
             for (int t = 0; t < 4; ++t) mx[t] = ptx::max3(mx[t], s[c + 2 * t], s[c + 2 * t + 1]);
           }
@@ -496,9 +530,15 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            float x0, x1;
+            float x0, x1, p0, p1;
             ptx::fma2(x0, x1, s[2 * c], s[2 * c + 1], sl, sl, neg_m, neg_m);
-            const uint32_t w2 = ptx::pack_bf16x2(ptx::ex2(x0), ptx::ex2(x1));
+            if (c % kPolyEvery == kPolyEvery - 1) {
+              exp2_poly2(p0, p1, x0, x1);
+            } else {
+              p0 = ptx::ex2(x0);
+              p1 = ptx::ex2(x1);
+            }
+            const uint32_t w2 = ptx::pack_bf16x2(p0, p1);
             pk[c >> 5][c & 31] = w2;
             ptx::add_bf16x2(ls[2 * (c & 1)], ls[2 * (c & 1) + 1], w2);
           }

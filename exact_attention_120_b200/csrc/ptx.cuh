@@ -224,6 +224,17 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
+// (a0, a1) + (b0, b1) as one packed two-lane fp32 add.
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 y, {%4, %5};\n\t"
+      "add.rn.f32x2 x, x, y;\n\t"
+      "mov.b64 {%0, %1}, x;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // acc_lo += float(bf16 bits [0,16) of w); acc_hi += float(bf16 bits [16,32) of w).
 // The bf16 -> fp32 widening is exact, so this sums the rounded values.
 __device__ __forceinline__ void add_bf16x2(float& acc_lo, float& acc_hi, uint32_t w) {

@@ -63,11 +63,19 @@ def full_parity(q, k, v, causal=False, mask=None, scale=None):
     return assert_parity(o, lse, o_ref, lse_ref)
 
 
-def sample_rows(B, H, N, count, seed):
-    """(b, h, i) samples: first and last rows, tile edges, and random rows."""
+def sample_rows(B, H, N, count, seed, per_tile=True):
+    """(b, h, i) samples: first and last rows, tile edges, one random row in
+    every (b, h, 128-row query tile) when `per_tile`, and random rows up to
+    `count` extra."""
     r = np.random.default_rng(seed)
     rows = {(0, 0, 0), (B - 1, H - 1, N - 1), (0, H - 1, min(N - 1, 127)),
             (B - 1, 0, min(N - 1, 128)), (0, 0, N // 2)}
-    while len(rows) < count:
+    if per_tile:
+        for b in range(B):
+            for h in range(H):
+                for t0 in range(0, N, 128):
+                    rows.add((b, h, int(r.integers(t0, min(N, t0 + 128)))))
+    target = len(rows) + count
+    while len(rows) < target:
         rows.add((int(r.integers(B)), int(r.integers(H)), int(r.integers(N))))
     return sorted(rows)
