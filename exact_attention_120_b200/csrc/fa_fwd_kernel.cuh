@@ -88,8 +88,9 @@ struct Cfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
-  // q_full, q_empty, full[S], empty[S], s_full[2], p_full[2], o_full[2], o_empty[2], mma_done
-  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  // q_full, q_empty, full[S], empty[S], s_full[2], p_full[2], o_full[2], o_empty[2],
+  // p_half[2], mma_done
+  static constexpr int kNumBars = 2 + 2 * kStages + 11;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 384;
@@ -194,13 +195,15 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
 
 // Barrier addresses shared by the kernel and the MMA helpers.  Layout from
 // bar0: q_full, q_empty, full[S], empty[S], s_full[2], p_full[2], o_full[2],
-// o_empty[2], mma_done.
+// o_empty[2], p_half[2], mma_done.
 template <int D> __device__ __forceinline__ uint32_t bar_full(uint32_t bar0, int s) { return bar0 + 16 + 8u * s; }
 template <int D> __device__ __forceinline__ uint32_t bar_q(uint32_t bar0) { return bar0 + 16 + 16u * Cfg<D>::kStages; }
 template <int D> __device__ __forceinline__ uint32_t bar_s_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 8u * q; }
 template <int D> __device__ __forceinline__ uint32_t bar_p_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 16 + 8u * q; }
 template <int D> __device__ __forceinline__ uint32_t bar_o_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 32 + 8u * q; }
 template <int D> __device__ __forceinline__ uint32_t bar_o_empty(uint32_t bar0, int q) { return bar_q<D>(bar0) + 48 + 8u * q; }
+// P of keys [0, 64) of the tile is in tensor memory (p_full: all 128 keys).
+template <int D> __device__ __forceinline__ uint32_t bar_p_half(uint32_t bar0, int q) { return bar_q<D>(bar0) + 64 + 8u * q; }
 
 // MMA-issuer state of one query slot.
 struct MmaSlot {
@@ -232,8 +235,8 @@ __device__ __forceinline__ bool mma_issue_pv(const MmaCtx<D>& c, const KernelPar
                                              int64_t& v_ready, uint32_t bar0) {
   using C = Cfg<D>;
   constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
-  if (!wait_warp(bar_p_full<D>(bar0, Q), s.pwait & 1u, c.abort_flag, p)) return false;
-  ++s.pwait;
+  // Keys [0, 64) of P first: their MMAs overlap the softmax of keys [64, 128).
+  if (!wait_warp(bar_p_half<D>(bar0, Q), s.pwait & 1u, c.abort_flag, p)) return false;
   ptx::tc_fence_after();
   const int64_t vr = s.pend;
   if (vr > v_ready) {
@@ -253,10 +256,18 @@ __device__ __forceinline__ bool mma_issue_pv(const MmaCtx<D>& c, const KernelPar
   const uint32_t tP = c.tmem + (Q ? C::kTmemS1 : C::kTmemS0);
   const uint32_t acc0 = s.npv > 0 ? 1u : 0u;
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk)
+  for (int kk = 0; kk < kBN / 32; ++kk)
     if (ptx::elect_one())
       ptx::mma_ts(tO, tP + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::kBoxBytes, 1024), kIdescPV,
                   kk > 0 ? 1u : acc0);
+  if (!wait_warp(bar_p_full<D>(bar0, Q), s.pwait & 1u, c.abort_flag, p)) return false;
+  ++s.pwait;
+  ptx::tc_fence_after();
+#pragma unroll
+  for (int kk = kBN / 32; kk < kBN / 16; ++kk)
+    if (ptx::elect_one())
+      ptx::mma_ts(tO, tP + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::kBoxBytes, 1024), kIdescPV,
+                  1u);
   ++s.npv;
   s.pend = -1;
   return true;
@@ -303,7 +314,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   auto bPFull = [&](int q) { return bar_p_full<D>(bar0, q); };
   auto bOFull = [&](int q) { return bar_o_full<D>(bar0, q); };
   auto bOEmpty = [&](int q) { return bar_o_empty<D>(bar0, q); };
-  const uint32_t bMmaDone = bar_q<D>(bar0) + 64;
+  auto bPHalf = [&](int q) { return bar_p_half<D>(bar0, q); };
+  const uint32_t bMmaDone = bar_q<D>(bar0) + 80;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kOffMisc + 4);
 
@@ -322,6 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       ptx::mbar_init(bPFull(q), 128);
       ptx::mbar_init(bOFull(q), 1);
       ptx::mbar_init(bOEmpty(q), 128);
+      ptx::mbar_init(bPHalf(q), 128);
     }
     ptx::mbar_init(bMmaDone, 1);
     *abort_flag = 0;
@@ -526,39 +539,50 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             m_ref = m_new;
           }
           const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-          uint32_t pk[2][32];
           float ls[4] = {0.f, 0.f, 0.f, 0.f};
+          // Keys [0, 64) then [64, 128): each half of P is stored and signalled
+          // as soon as it exists, so the PV MMAs of the first half overlap the
+          // exponentials of the second.
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            float x0, x1, p0, p1;
-            ptx::fma2(x0, x1, s[2 * c], s[2 * c + 1], sl, sl, neg_m, neg_m);
-            if (c % kPolyEvery == kPolyEvery - 1) {
-              exp2_poly2(p0, p1, x0, x1);
-            } else {
-              p0 = ptx::ex2(x0);
-              p1 = ptx::ex2(x1);
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int cc = 32 * half + c;
+              float x0, x1, p0, p1;
+              ptx::fma2(x0, x1, s[2 * cc], s[2 * cc + 1], sl, sl, neg_m, neg_m);
+              if (cc % kPolyEvery == kPolyEvery - 1) {
+                exp2_poly2(p0, p1, x0, x1);
+              } else {
+                p0 = ptx::ex2(x0);
+                p1 = ptx::ex2(x1);
+              }
+              const uint32_t w2 = ptx::pack_bf16x2(p0, p1);
+              pk[c] = w2;
+              ptx::add_bf16x2(ls[2 * (c & 1)], ls[2 * (c & 1) + 1], w2);
             }
-            const uint32_t w2 = ptx::pack_bf16x2(p0, p1);
-            pk[c >> 5][c & 31] = w2;
-            ptx::add_bf16x2(ls[2 * (c & 1)], ls[2 * (c & 1) + 1], w2);
+            ptx::tmem_st32(tS + 32 * half, pk);
+            if (half == 0) {
+              // O holds earlier tiles: rescale it in place before any PV of this
+              // tile.  tcgen05.ld/st are warp-collective, so the warp rescales
+              // together (alpha = 1 for rows whose reference did not move).
+              if (n > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                  uint32_t t[32];
+                  ptx::tmem_ld32(tO + 32 * c, t);
+                  ptx::tmem_wait_ld();
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
+                  ptx::tmem_st32(tO + 32 * c, t);
+                }
+              }
+              ptx::tmem_wait_st();
+              ptx::tc_fence_before();
+              ptx::mbar_arrive(bPHalf(q));
+            }
           }
           l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-          ptx::tmem_st32(tS, pk[0]);
-          ptx::tmem_st32(tS + 32, pk[1]);
-          // O holds earlier tiles: rescale it in place.  tcgen05.ld/st are
-          // warp-collective, so the warp rescales together (alpha = 1 for rows
-          // whose reference did not move).
-          if (n > 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t t[32];
-              ptx::tmem_ld32(tO + 32 * c, t);
-              ptx::tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) t[e] = __float_as_uint(__uint_as_float(t[e]) * alpha);
-              ptx::tmem_st32(tO + 32 * c, t);
-            }
-          }
           ptx::tmem_wait_st();
           ptx::tc_fence_before();
           ptx::mbar_arrive(bPFull(q));
