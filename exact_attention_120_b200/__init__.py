@@ -49,6 +49,9 @@ _SIGNATURES = {
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_cuda_error": (ctypes.c_int, []),
     "fa_launches_per_call": (ctypes.c_int, []),
+    "fa_testing_fwd_starved": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
+                               + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                                       ctypes.c_void_p, ctypes.c_ulonglong]),
 }
 
 

@@ -22,7 +22,7 @@ LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 SOURCES = [os.path.join(CSRC, "fa_api.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "ptx.cuh")] + [
-    os.path.join(INCLUDE, "fa.h")]
+    os.path.join(INCLUDE, "fa.h"), os.path.join(INCLUDE, "fa_testing.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

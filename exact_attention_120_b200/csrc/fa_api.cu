@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_testing.h"
 #include "fa_fwd_kernel.cuh"
 
 namespace {
@@ -119,13 +120,10 @@ int encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
   return FA_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-                  int N, int d, float scale, int causal, const uint8_t* block_mask,
-                  void* cuda_stream) {
+// Validation, descriptors and launch shared by the entry points.
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int N, int d, float scale, int causal, const uint8_t* block_mask, void* cuda_stream,
+               unsigned long long timeout_ns, int starve_producer) {
   // ---- arguments (nothing is launched on error)
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARGUMENT;
@@ -166,8 +164,9 @@ int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, float* l
   p.items = (int)(bh * npairs);
   p.causal = causal;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
-  p.timeout_ns = kWaitTimeoutNs;
+  p.timeout_ns = timeout_ns;
   p.status = st->status_word;
+  p.starve_producer = starve_producer;
 
   // ---- launch: persistent grid, one CTA per SM
   const int grid = p.items < st->num_sms ? p.items : st->num_sms;
@@ -179,6 +178,26 @@ int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, float* l
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                  int N, int d, float scale, int causal, const uint8_t* block_mask,
+                  void* cuda_stream) {
+  return launch_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, cuda_stream,
+                    kWaitTimeoutNs, 0);
+}
+
+int fa_testing_fwd_starved(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int H, int N, int d, float scale, int causal,
+                           const uint8_t* block_mask, void* cuda_stream,
+                           unsigned long long timeout_ns) {
+  if (timeout_ns == 0 || timeout_ns > kWaitTimeoutNs) return FA_ERR_INVALID_ARGUMENT;
+  return launch_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, cuda_stream,
+                    timeout_ns, 1);
 }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,

@@ -76,6 +76,10 @@ struct KernelParams {
   float scale_log2;  // scale * log2(e)
   unsigned long long timeout_ns;
   int* status;  // device status word
+  // Test hook of the failure-detection test: when set, the TMA producer issues
+  // nothing, so the first barrier wait of the MMA issuer can never complete and
+  // must end through its time limit.  Always 0 on the production entry points.
+  int starve_producer;
 };
 
 template <int D>
@@ -360,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     uint32_t it = 0;       // K/V ring loads issued
     uint32_t nq = 0;       // Q loads issued
     bool ok = true;
-    for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
+    for (int w = blockIdx.x; w < p.items && ok && !p.starve_producer; w += gridDim.x) {
       int bh, pair;
       decode_item(p, w, bh, pair);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
