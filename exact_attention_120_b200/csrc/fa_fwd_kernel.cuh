@@ -93,11 +93,18 @@ struct Cfg {
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
   // q_full, q_empty, full[S], empty[S], s_full[2], p_full[2], o_full[2], o_empty[2],
-  // p_half[2], mma_done
-  static constexpr int kNumBars = 2 + 2 * kStages + 11;
+  // p_half[2], s_free[2], pv_done[2], mma_done
+  static constexpr int kNumBars = 2 + 2 * kStages + 15;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
-  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256, kTmemO1 = 384;
+  // Tensor memory columns.  At d = 128, S_0, S_1, O_0, O_1 fill all 512 and P_q
+  // is written over S_q.  At d = 64 there is room for P_q of its own, so the
+  // next S_q can be computed while the softmax of the current one still runs.
+  static constexpr bool kSeparateP = (D == 64);
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256;
+  static constexpr uint32_t kTmemO1 = kSeparateP ? 320 : 384;
+  static constexpr uint32_t kTmemP0 = kSeparateP ? 384 : kTmemS0;
+  static constexpr uint32_t kTmemP1 = kSeparateP ? 448 : kTmemS1;
 };
 
 // 2^x on the FMA pipe for two lanes (relieves the MUFU exp2 unit, which at
@@ -208,6 +215,11 @@ template <int D> __device__ __forceinline__ uint32_t bar_o_full(uint32_t bar0, i
 template <int D> __device__ __forceinline__ uint32_t bar_o_empty(uint32_t bar0, int q) { return bar_q<D>(bar0) + 48 + 8u * q; }
 // P of keys [0, 64) of the tile is in tensor memory (p_full: all 128 keys).
 template <int D> __device__ __forceinline__ uint32_t bar_p_half(uint32_t bar0, int q) { return bar_q<D>(bar0) + 64 + 8u * q; }
+// Separate-P layout only: the softmax has read S_q (s_free), the PV MMAs of
+// slot q's latest P are complete (pv_done).
+template <int D> __device__ __forceinline__ uint32_t bar_s_free(uint32_t bar0, int q) { return bar_q<D>(bar0) + 80 + 8u * q; }
+template <int D> __device__ __forceinline__ uint32_t bar_pv_done(uint32_t bar0, int q) { return bar_q<D>(bar0) + 96 + 8u * q; }
+template <int D> __device__ __forceinline__ uint32_t bar_mma_done(uint32_t bar0) { return bar_q<D>(bar0) + 112; }
 
 // MMA-issuer state of one query slot.
 struct MmaSlot {
@@ -215,6 +227,7 @@ struct MmaSlot {
   uint32_t npv = 0;      // PV MMAs issued in this work unit
   uint32_t pwait = 0;    // p_full phases consumed
   uint32_t nitems = 0;   // work units seen with this slot valid
+  uint32_t ns = 0;       // S MMAs issued (separate-P layout: s_free phases owed)
   bool need_oe = false;  // must wait for the previous unit's epilogue first
   __device__ __forceinline__ void begin_unit(bool valid) {
     pend = -1;
@@ -257,7 +270,7 @@ __device__ __forceinline__ bool mma_issue_pv(const MmaCtx<D>& c, const KernelPar
   }
   const uint32_t vbase = c.sRing + (uint32_t)(vr % C::kStages) * C::kTileBytes;
   const uint32_t tO = c.tmem + (Q ? C::kTmemO1 : C::kTmemO0);
-  const uint32_t tP = c.tmem + (Q ? C::kTmemS1 : C::kTmemS0);
+  const uint32_t tP = c.tmem + (Q ? C::kTmemP1 : C::kTmemP0);
   const uint32_t acc0 = s.npv > 0 ? 1u : 0u;
 #pragma unroll
   for (int kk = 0; kk < kBN / 32; ++kk)
@@ -272,19 +285,23 @@ __device__ __forceinline__ bool mma_issue_pv(const MmaCtx<D>& c, const KernelPar
     if (ptx::elect_one())
       ptx::mma_ts(tO, tP + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::kBoxBytes, 1024), kIdescPV,
                   1u);
+  if (C::kSeparateP && ptx::elect_one()) ptx::mma_commit(bar_pv_done<D>(bar0, Q));
   ++s.npv;
   s.pend = -1;
   return true;
 }
 
-// One kept K tile for slot Q: settle its pending PV, then S_q = Q_q K_j^T.
-// Warp-uniform, like mma_issue_pv.
+// S_q = Q_q K_j^T into slot Q's S columns (warp-uniform).  With the
+// separate-P layout the softmax must first have read the previous S_q.
 template <int D, int Q>
-__device__ __forceinline__ bool mma_slot_step(const MmaCtx<D>& c, const KernelParams& p, MmaSlot& s,
-                                              int64_t& v_ready, int kslot, uint32_t vr, uint32_t bar0) {
+__device__ __forceinline__ bool mma_issue_s(const MmaCtx<D>& c, const KernelParams& p, MmaSlot& s,
+                                            int kslot, uint32_t bar0) {
   using C = Cfg<D>;
   constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
-  if (s.pend >= 0 && !mma_issue_pv<D, Q>(c, p, s, v_ready, bar0)) return false;
+  if (C::kSeparateP && s.ns > 0) {
+    if (!wait_warp(bar_s_free<D>(bar0, Q), (s.ns - 1) & 1u, c.abort_flag, p)) return false;
+    ptx::tc_fence_after();
+  }
   const uint32_t qbase = c.sQ + Q * C::kTileBytes;
   const uint32_t kbase = c.sRing + kslot * C::kTileBytes;
   const uint32_t tS = c.tmem + (Q ? C::kTmemS1 : C::kTmemS0);
@@ -296,6 +313,17 @@ __device__ __forceinline__ bool mma_slot_step(const MmaCtx<D>& c, const KernelPa
                   kIdescQK, kk > 0 ? 1u : 0u);
   }
   if (ptx::elect_one()) ptx::mma_commit(bar_s_full<D>(bar0, Q));
+  ++s.ns;
+  return true;
+}
+
+// One kept K tile for slot Q in the P-over-S layout: settle its pending PV
+// (P_q shares columns with S_q), then S_q = Q_q K_j^T.  Warp-uniform.
+template <int D, int Q>
+__device__ __forceinline__ bool mma_slot_step(const MmaCtx<D>& c, const KernelParams& p, MmaSlot& s,
+                                              int64_t& v_ready, int kslot, uint32_t vr, uint32_t bar0) {
+  if (s.pend >= 0 && !mma_issue_pv<D, Q>(c, p, s, v_ready, bar0)) return false;
+  if (!mma_issue_s<D, Q>(c, p, s, kslot, bar0)) return false;
   s.pend = vr;
   return true;
 }
@@ -319,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   auto bOFull = [&](int q) { return bar_o_full<D>(bar0, q); };
   auto bOEmpty = [&](int q) { return bar_o_empty<D>(bar0, q); };
   auto bPHalf = [&](int q) { return bar_p_half<D>(bar0, q); };
-  const uint32_t bMmaDone = bar_q<D>(bar0) + 80;
+  const uint32_t bMmaDone = bar_mma_done<D>(bar0);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kOffMisc + 4);
 
@@ -339,6 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       ptx::mbar_init(bOFull(q), 1);
       ptx::mbar_init(bOEmpty(q), 128);
       ptx::mbar_init(bPHalf(q), 128);
+      ptx::mbar_init(bar_s_free<D>(bar0, q), 128);
+      ptx::mbar_init(bar_pv_done<D>(bar0, q), 1);
     }
     ptx::mbar_init(bMmaDone, 1);
     *abort_flag = 0;
@@ -441,15 +471,27 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           ok = wait_warp(bFull(kslot), (kr / C::kStages) & 1u, abort_flag, p);
           ptx::tc_fence_after();
           const bool keep0 = ((k0 >> l) & 1u) != 0, keep1 = ((k1 >> l) & 1u) != 0;
-          // Slot q: pending O_q += P_q V first (P_q shares columns with S_q),
-          // then S_q = Q_q K_j^T.
-          if (ok && keep0) ok = mma_slot_step<D, 0>(ctx, p, slot0, v_ready, kslot, vr, bar0);
-          if (ok && keep1) ok = mma_slot_step<D, 1>(ctx, p, slot1, v_ready, kslot, vr, bar0);
-          if (ok && ptx::elect_one()) ptx::mma_commit(bEmpty(kslot));  // K_j no longer needed
-          // A slot that skips K_j still owes a PV on the previous V: issue it
-          // now so that V can be released.
-          if (ok && !keep0 && slot0.pend >= 0) ok = mma_issue_pv<D, 0>(ctx, p, slot0, v_ready, bar0);
-          if (ok && !keep1 && slot1.pend >= 0) ok = mma_issue_pv<D, 1>(ctx, p, slot1, v_ready, bar0);
+          if constexpr (C::kSeparateP) {
+            // Both S first (the softmax has already read the previous S), then
+            // the PVs of the previous tile, whose P lives in its own columns.
+            if (ok && keep0) ok = mma_issue_s<D, 0>(ctx, p, slot0, kslot, bar0);
+            if (ok && keep1) ok = mma_issue_s<D, 1>(ctx, p, slot1, kslot, bar0);
+            if (ok && ptx::elect_one()) ptx::mma_commit(bEmpty(kslot));  // K_j no longer needed
+            if (ok && slot0.pend >= 0) ok = mma_issue_pv<D, 0>(ctx, p, slot0, v_ready, bar0);
+            if (ok && slot1.pend >= 0) ok = mma_issue_pv<D, 1>(ctx, p, slot1, v_ready, bar0);
+            if (keep0) slot0.pend = vr;
+            if (keep1) slot1.pend = vr;
+          } else {
+            // Slot q: pending O_q += P_q V first (P_q shares columns with S_q),
+            // then S_q = Q_q K_j^T.
+            if (ok && keep0) ok = mma_slot_step<D, 0>(ctx, p, slot0, v_ready, kslot, vr, bar0);
+            if (ok && keep1) ok = mma_slot_step<D, 1>(ctx, p, slot1, v_ready, kslot, vr, bar0);
+            if (ok && ptx::elect_one()) ptx::mma_commit(bEmpty(kslot));  // K_j no longer needed
+            // A slot that skips K_j still owes a PV on the previous V: issue it
+            // now so that V can be released.
+            if (ok && !keep0 && slot0.pend >= 0) ok = mma_issue_pv<D, 0>(ctx, p, slot0, v_ready, bar0);
+            if (ok && !keep1 && slot1.pend >= 0) ok = mma_issue_pv<D, 1>(ctx, p, slot1, v_ready, bar0);
+          }
           if (ok && prev_v >= 0 && ptx::elect_one())
             ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
           prev_v = vr;
@@ -482,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_base + (q ? C::kTmemS1 : C::kTmemS0);
     const uint32_t tO = tmem + lane_base + (q ? C::kTmemO1 : C::kTmemO0);
+    const uint32_t tP = tmem + lane_base + (q ? C::kTmemP1 : C::kTmemP0);
     const float sl = p.scale_log2;
     uint32_t swait = 0, owait = 0;
     bool ok = true;
@@ -508,6 +551,10 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
 #pragma unroll
           for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, r[c]);
           ptx::tmem_wait_ld();
+          if constexpr (C::kSeparateP) {  // S_q may now be overwritten by the next tile
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar_s_free<D>(bar0, q));
+          }
           float s[128];
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c >> 5][c & 31]);
@@ -543,6 +590,14 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             m_ref = m_new;
           }
           const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          if constexpr (C::kSeparateP) {
+            // P_q and O_q are still read / written by the previous tile's PV.
+            if (swait >= 2) {
+              ok = wait_warp(bar_pv_done<D>(bar0, q), (swait - 2) & 1u, abort_flag, p);
+              if (!ok) break;
+              ptx::tc_fence_after();
+            }
+          }
           float ls[4] = {0.f, 0.f, 0.f, 0.f};
           // Keys [0, 64) then [64, 128): each half of P is stored and signalled
           // as soon as it exists, so the PV MMAs of the first half overlap the
@@ -565,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
               pk[c] = w2;
               ptx::add_bf16x2(ls[2 * (c & 1)], ls[2 * (c & 1) + 1], w2);
             }
-            ptx::tmem_st32(tS + 32 * half, pk);
+            ptx::tmem_st32(tP + 32 * half, pk);
             if (half == 0) {
               // O holds earlier tiles: rescale it in place before any PV of this
               // tile.  tcgen05.ld/st are warp-collective, so the warp rescales
