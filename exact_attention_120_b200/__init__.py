@@ -9,6 +9,7 @@ Functions with the C names take raw device addresses:
 
 * ``fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask)``
 * ``fa_fwd_stream(..., stream)``
+* ``fa_fwd_qk(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, stream)``
 * ``fa_device_status(stream)``, ``fa_status_string(status)``
 
 and ``attention_forward(q, k, v, ...)`` is the tensor-level convenience that
@@ -22,7 +23,8 @@ import math
 import os
 
 __all__ = [
-    "FaError", "library_path", "load_library", "fa_fwd", "fa_fwd_stream", "fa_device_status",
+    "FaError", "library_path", "load_library", "fa_fwd", "fa_fwd_stream", "fa_fwd_qk",
+    "fa_device_status",
     "fa_status_string", "fa_launches_per_call", "attention_forward", "FA_OK",
     "FA_ERR_INVALID_ARGUMENT", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT",
     "MASK_BLOCK",
@@ -45,6 +47,9 @@ _SIGNATURES = {
     "fa_fwd_stream": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
                       + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                               ctypes.c_void_p]),
+    "fa_fwd_qk": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
+                  + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_void_p]),
     "fa_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_cuda_error": (ctypes.c_int, []),
@@ -97,6 +102,12 @@ def fa_fwd_stream(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, stream
                                         stream)
 
 
+def fa_fwd_qk(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, stream) -> int:
+    """C ``fa_fwd_qk`` (Nq query rows, Nk keys) on raw device addresses."""
+    return load_library().fa_fwd_qk(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask,
+                                    stream)
+
+
 def fa_device_status(stream=None) -> int:
     return load_library().fa_device_status(stream)
 
@@ -111,38 +122,48 @@ def fa_launches_per_call() -> int:
 
 def attention_forward(q, k, v, causal=False, block_mask=None, scale=None, out=None, lse=None,
                       stream=None):
-    """O, lse = attention(q, k, v) through ``fa_fwd_stream``.
+    """O, lse = attention(q, k, v) through the C ABI.
 
-    q, k, v: CUDA bfloat16 tensors [B, H, N, d], contiguous, d in {64, 128}.
-    block_mask: None or a CUDA uint8 tensor [B, H, ceil(N/128), ceil(N/128)].
-    scale: defaults to 1/sqrt(d).  Returns (o bf16 [B,H,N,d], lse fp32 [B,H,N]).
+    q: CUDA bfloat16 [B, H, Nq, d]; k, v: CUDA bfloat16 [B, H, Nk, d]; all
+    contiguous, d in {64, 128}.  Nq = Nk uses ``fa_fwd_stream``, otherwise
+    ``fa_fwd_qk`` (causal diagonal aligned to the last key).
+    block_mask: None or a CUDA uint8 tensor [B, H, ceil(Nq/128), ceil(Nk/128)].
+    scale: defaults to 1/sqrt(d).  Returns (o bf16 [B,H,Nq,d], lse fp32 [B,H,Nq]).
     """
     import torch
 
-    if q.dim() != 4 or q.shape != k.shape or q.shape != v.shape:
-        raise ValueError("q, k, v must share one [B, H, N, d] shape")
+    if q.dim() != 4 or k.shape != v.shape or k.dim() != 4 or q.shape[:2] != k.shape[:2] \
+            or q.shape[3] != k.shape[3]:
+        raise ValueError("q must be [B, H, Nq, d] and k, v [B, H, Nk, d]")
     for t in (q, k, v):
         if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
             raise ValueError("q, k, v must be contiguous CUDA bfloat16 tensors")
-    B, H, N, d = q.shape
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
     mask_ptr = None
     if block_mask is not None:
-        nb = (N + MASK_BLOCK - 1) // MASK_BLOCK
+        nbq = (Nq + MASK_BLOCK - 1) // MASK_BLOCK
+        nbk = (Nk + MASK_BLOCK - 1) // MASK_BLOCK
         if (block_mask.dtype != torch.uint8 or not block_mask.is_cuda
-                or tuple(block_mask.shape) != (B, H, nb, nb) or not block_mask.is_contiguous()):
-            raise ValueError(f"block_mask must be a contiguous CUDA uint8 [B,H,{nb},{nb}] tensor")
+                or tuple(block_mask.shape) != (B, H, nbq, nbk) or not block_mask.is_contiguous()):
+            raise ValueError(f"block_mask must be a contiguous CUDA uint8 [B,H,{nbq},{nbk}] tensor")
         mask_ptr = block_mask.data_ptr()
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     with torch.cuda.device(q.device):
-        st = fa_fwd_stream(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                           B, H, N, d, float(scale), int(bool(causal)), mask_ptr, stream)
+        if Nq == Nk:
+            st = fa_fwd_stream(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), B, H, Nq, d, float(scale), int(bool(causal)),
+                               mask_ptr, stream)
+        else:
+            st = fa_fwd_qk(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                           B, H, Nq, Nk, d, float(scale), int(bool(causal)), mask_ptr, stream)
     if st != FA_OK:
-        raise FaError(st, "fa_fwd_stream")
+        raise FaError(st, "fa_fwd")
     return out, lse

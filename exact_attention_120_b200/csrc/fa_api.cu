@@ -122,20 +122,22 @@ int encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
 
 // Validation, descriptors and launch shared by the entry points.
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int N, int d, float scale, int causal, const uint8_t* block_mask, void* cuda_stream,
-               unsigned long long timeout_ns, int starve_producer) {
+               int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
+               void* cuda_stream, unsigned long long timeout_ns, int starve_producer) {
   // ---- arguments (nothing is launched on error)
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
-  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARGUMENT;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARGUMENT;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARGUMENT;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_INVALID_ARGUMENT;
   const long long bh = (long long)B * H;
-  const long long nqt = (N + fa::kBM - 1) / fa::kBM;
+  const long long nqt = (Nq + fa::kBM - 1) / fa::kBM;
+  const long long nkt = (Nk + fa::kBN - 1) / fa::kBN;
   const long long npairs = (nqt + 1) / 2;
-  if (bh > INT32_MAX || bh * npairs > INT32_MAX || (long long)N * d * 2 >= (1ll << 40))
+  if (bh > INT32_MAX || bh * npairs > INT32_MAX || (long long)Nq * d * 2 >= (1ll << 40) ||
+      (long long)Nk * d * 2 >= (1ll << 40))
     return FA_ERR_UNSUPPORTED;  // 32-bit work indices and TMA stride limits
   if (o == q || o == k || o == v) return FA_ERR_INVALID_ARGUMENT;
 
@@ -151,14 +153,17 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   // ---- parameters
   fa::KernelParams p;
   std::memset(&p, 0, sizeof(p));
-  if ((rc = encode_qkv_map(&p.tm_q, q, (int)bh, N, d)) != FA_OK) return rc;
-  if ((rc = encode_qkv_map(&p.tm_k, k, (int)bh, N, d)) != FA_OK) return rc;
-  if ((rc = encode_qkv_map(&p.tm_v, v, (int)bh, N, d)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_q, q, (int)bh, Nq, d)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_k, k, (int)bh, Nk, d)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_v, v, (int)bh, Nk, d)) != FA_OK) return rc;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.mask = block_mask;
-  p.N = N;
+  p.Nq = Nq;
+  p.Nk = Nk;
   p.nqt = (int)nqt;
+  p.nkt = (int)nkt;
+  p.causal_off = Nk - Nq;
   p.npairs = (int)npairs;
   p.bh = (int)bh;
   p.items = (int)(bh * npairs);
@@ -187,7 +192,14 @@ extern "C" {
 int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                   int N, int d, float scale, int causal, const uint8_t* block_mask,
                   void* cuda_stream) {
-  return launch_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, cuda_stream,
+  return launch_fwd(q, k, v, o, lse, B, H, N, N, d, scale, causal, block_mask, cuda_stream,
+                    kWaitTimeoutNs, 0);
+}
+
+int fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+              int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
+              void* cuda_stream) {
+  return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
                     kWaitTimeoutNs, 0);
 }
 
@@ -196,7 +208,7 @@ int fa_testing_fwd_starved(const void* q, const void* k, const void* v, void* o,
                            const uint8_t* block_mask, void* cuda_stream,
                            unsigned long long timeout_ns) {
   if (timeout_ns == 0 || timeout_ns > kWaitTimeoutNs) return FA_ERR_INVALID_ARGUMENT;
-  return launch_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, cuda_stream,
+  return launch_fwd(q, k, v, o, lse, B, H, N, N, d, scale, causal, block_mask, cuda_stream,
                     timeout_ns, 1);
 }
 

@@ -66,10 +66,13 @@ struct KernelParams {
   CUtensorMap tm_v;
   __nv_bfloat16* o;
   float* lse;
-  const uint8_t* mask;  // nullptr or [B*H][nqt][nqt]
-  int N;
-  int nqt;     // query (= key) tiles per head
-  int npairs;  // work units per head
+  const uint8_t* mask;  // nullptr or [B*H][nqt][nkt]
+  int Nq;          // query rows per head
+  int Nk;          // keys per head
+  int nqt;         // query tiles per head
+  int nkt;         // key tiles per head
+  int causal_off;  // Nk - Nq: key j is visible to query i iff j <= i + causal_off
+  int npairs;      // work units per head
   int bh;      // B * H
   int items;   // bh * npairs
   int causal;
@@ -167,13 +170,26 @@ __device__ __forceinline__ void decode_item(const KernelParams& p, int w, int& b
   }
 }
 
+// Largest key index query tile qt can see under the causal rule (may be < 0).
+__device__ __forceinline__ int causal_last_key(const KernelParams& p, int qt) {
+  return min(qt * kBM + kBM - 1, p.Nq - 1) + p.causal_off;
+}
+
+// Number of key tiles to scan for query tile qt: all of them, or under the
+// causal rule those up to the tile of its last visible key.
+__device__ __forceinline__ int key_tile_end(const KernelParams& p, int qt) {
+  if (!p.causal) return p.nkt;
+  const int last = causal_last_key(p, qt);
+  return last < 0 ? 0 : min(p.nkt, last / kBN + 1);
+}
+
 // Bit l set <=> key tile j0 + l is visible to query tile qt (whole warp calls).
 __device__ __forceinline__ uint32_t keep_bits(const KernelParams& p, int bh, int qt, int j0,
                                               int lane) {
   const int j = j0 + lane;
-  bool k = (qt < p.nqt) && (j < p.nqt);
-  if (k && p.causal) k = (j <= qt);
-  if (k && p.mask != nullptr) k = p.mask[((size_t)bh * p.nqt + qt) * p.nqt + j] != 0;
+  bool k = (qt < p.nqt) && (j < p.nkt);
+  if (k && p.causal) k = j * kBN <= causal_last_key(p, qt);
+  if (k && p.mask != nullptr) k = p.mask[((size_t)bh * p.nqt + qt) * p.nkt + j] != 0;
   return __ballot_sync(0xffffffffu, k);
 }
 
@@ -408,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
                              (qt0 + q) * kBM, bh);
       }
       ++nq;
-      const int jend = p.causal ? min(p.nqt, qt0 + nvalid) : p.nqt;
+      const int jend = key_tile_end(p, qt0 + nvalid - 1);
       for (int j0 = 0; j0 < jend && ok; j0 += 32) {
         uint32_t u = keep_bits(p, bh, qt0, j0, lane) | keep_bits(p, bh, qt1, j0, lane);
         while (u != 0 && ok) {
@@ -457,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       ok = wait_warp(bQFull, nq & 1u, abort_flag, p);
       ptx::tc_fence_after();
       ++nq;
-      const int jend = p.causal ? min(p.nqt, qt0 + (valid1 ? 2 : 1)) : p.nqt;
+      const int jend = key_tile_end(p, valid1 ? qt1 : qt0);
       for (int j0 = 0; j0 < jend && ok; j0 += 32) {
         const uint32_t k0 = keep_bits(p, bh, qt0, j0, lane);
         const uint32_t k1 = keep_bits(p, bh, qt1, j0, lane);
@@ -533,11 +549,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       decode_item(p, w, bh, pair);
       const int qt = 2 * pair + q;
       if (qt >= p.nqt) continue;
-      const int row = qt * kBM + row_in_tile;
+      const int row = qt * kBM + row_in_tile;  // query row within the head
       float m_ref = -INFINITY;  // reference max, in units of c * score
       float l = 0.f;            // sum of bf16-rounded 2^(c s - m_ref)
       int n = 0;                // tiles processed
-      const int jend = p.causal ? min(p.nqt, qt + 1) : p.nqt;
+      const int jend = key_tile_end(p, qt);
       for (int j0 = 0; j0 < jend && ok; j0 += 32) {
         uint32_t kb = keep_bits(p, bh, qt, j0, lane);
         while (kb != 0 && ok) {
@@ -558,11 +574,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           float s[128];
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(r[c >> 5][c & 31]);
-          // Mask: causal diagonal tile and the ragged tail of the sequence.
+          // Mask: keys past the causal diagonal and past the end of the
+          // sequence (lim = last visible column of this tile, may be < 0).
           int lim = 127;
-          if (p.causal && j == qt) lim = row_in_tile;
-          const int tail = p.N - j * kBN - 1;
-          if (tail < lim) lim = tail;
+          if (p.causal) lim = min(lim, row + p.causal_off - j * kBN);
+          lim = min(lim, p.Nk - j * kBN - 1);
           if (lim < 127) {
 #pragma unroll
             for (int c = 0; c < 128; ++c)
@@ -656,9 +672,12 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         if (!ok) break;
         ptx::tc_fence_after();
       }
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      const bool in_range = row < p.N;
-      uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)bh * p.N + (in_range ? row : 0)) * D);
+      // A row whose reference max never left -inf saw no visible key (masked
+      // scores only add 2^-125 through the FMA-pipe exp2): O = 0, lse = -inf.
+      const bool seen = m_ref != -INFINITY && l > 0.f;
+      const float inv = seen ? 1.f / l : 0.f;
+      const bool in_range = row < p.Nq;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t t[32];
@@ -682,8 +701,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       ptx::tc_fence_before();
       ptx::mbar_arrive(bOEmpty(q));
       if (in_range)
-        p.lse[(size_t)bh * p.N + row] =
-            (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        p.lse[(size_t)bh * p.Nq + row] =
+            seen ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
   }
 

@@ -84,6 +84,23 @@ FA_API int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, f
                   void* cuda_stream);
 
 /*
+ * Attention with Nq query rows and Nk keys per (b, h) -- cross-attention, or
+ * decoding against a key/value cache.  q, o: [B, H, Nq, d]; k, v: [B, H, Nk, d];
+ * lse: [B, H, Nq]; block_mask: NULL or [B, H, ceil(Nq/128), ceil(Nk/128)].
+ * With `causal`, key j is visible to query i iff j <= i + (Nk - Nq): the
+ * queries are the last Nq positions of the sequence (the diagonal is aligned
+ * to the last key; for Nq = Nk this is j <= i).  When Nq > Nk the first
+ * Nq - Nk rows see no key and get O = 0, lse = -inf.  Otherwise identical to
+ * fa_fwd_stream; fa_fwd_stream(..., N, ...) equals fa_fwd_qk(..., N, N, ...).
+ * The problem statement this generalises is the one of fa_fwd (scaled
+ * dot-product attention, "理解 Flash Attention" section "什么是注意力");
+ * different lengths and the causal alignment are this library's extension.
+ */
+FA_API int fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int Nq, int Nk, int d, float scale, int causal,
+                     const uint8_t* block_mask, void* cuda_stream);
+
+/*
  * Reads and clears the device-side status word of the current device after
  * synchronising `cuda_stream`.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT (a
  * kernel's wait on one of its own barriers exceeded the time limit; the

@@ -51,7 +51,9 @@ def _as64(a):
 def visible_mask(n_q, n_k, causal, block_mask_bh=None, block=MASK_BLOCK, rows=None):
     """Boolean [len(rows), n_k] visibility of keys for the given query rows.
 
-    causal: key j visible to query i iff j <= i.
+    causal: key j visible to query i iff j <= i + (n_k - n_q), i.e. the
+    diagonal is aligned to the last key (for n_q = n_k: j <= i; with fewer
+    queries than keys the queries are the latest positions of the sequence).
     block_mask_bh: [ceil(n_q/block), ceil(n_k/block)] array, nonzero = the
     block of (query block, key block) is kept.  Both rules intersect.
     """
@@ -61,7 +63,7 @@ def visible_mask(n_q, n_k, causal, block_mask_bh=None, block=MASK_BLOCK, rows=No
     cols = np.arange(n_k)
     vis = np.ones((rows.size, n_k), dtype=bool)
     if causal:
-        vis &= cols[None, :] <= rows[:, None]
+        vis &= cols[None, :] <= rows[:, None] + (n_k - n_q)
     if block_mask_bh is not None:
         bm = np.asarray(block_mask_bh) != 0
         vis &= bm[(rows // block)[:, None], (cols // block)[None, :]]
@@ -99,15 +101,15 @@ def _rows_of_head(qh, kh, vh, scale, causal, bm_bh, block, rows):
 
 
 def attention_ref(q, k, v, scale, causal=False, block_mask=None, block=MASK_BLOCK, row_chunk=1024):
-    """Full oracle: O [B,H,N,d] and lse [B,H,N], both float64.
+    """Full oracle: O [B,H,Nq,d] and lse [B,H,Nq], both float64.
 
-    q, k, v: [B, H, N, d] arrays (converted exactly to float64).
-    block_mask: None or [B, H, ceil(N/block), ceil(N/block)], nonzero = keep.
+    q: [B, H, Nq, d]; k, v: [B, H, Nk, d] (converted exactly to float64).
+    block_mask: None or [B, H, ceil(Nq/block), ceil(Nk/block)], nonzero = keep.
     Rows are processed ``row_chunk`` at a time; each chunk holds complete
     rows of S, so the result is the definition, never an online update.
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
-    B, H, N, d = q.shape
+    B, H, N, d = q.shape  # N query rows; k and v may hold a different number of keys
     o = np.zeros((B, H, N, v.shape[-1]), dtype=np.float64)
     lse = np.zeros((B, H, N), dtype=np.float64)
     for b in range(B):
@@ -155,6 +157,7 @@ def attention_tiled_online(q, k, v, scale, causal=False, block_mask=None, block=
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
     B, H, N, d = q.shape
+    Nk = k.shape[2]
     dv = v.shape[-1]
     o = np.zeros((B, H, N, dv))
     lse = np.zeros((B, H, N))
@@ -164,10 +167,10 @@ def attention_tiled_online(q, k, v, scale, causal=False, block_mask=None, block=
             for q0 in range(0, N, bm):
                 rows = np.arange(q0, min(N, q0 + bm))
                 state = [(-math.inf, 0.0, np.zeros(dv)) for _ in rows]
-                for k0 in range(0, N, bn):
-                    cols = np.arange(k0, min(N, k0 + bn))
+                for k0 in range(0, Nk, bn):
+                    cols = np.arange(k0, min(Nk, k0 + bn))
                     s = scale * (q[b, h, rows] @ k[b, h, cols].T)
-                    vis = visible_mask(N, N, causal, bmask, block, rows)[:, cols]
+                    vis = visible_mask(N, Nk, causal, bmask, block, rows)[:, cols]
                     s = np.where(vis, s, -np.inf)
                     for r in range(rows.size):
                         state[r] = merge_partials(state[r], partial_state(s[r], v[b, h, cols]))

@@ -8,7 +8,8 @@ arithmetic.  It computes, for every query row i of every (b, h),
     w_ij = exp(s_ij - max_j s_ij)
     O_i  = sum_j w_ij v_j / sum_j w_ij,   lse_i = max_j s_ij + ln(sum_j w_ij)
 
-with visibility j <= i when causal and the 128x128 (or ``block``-sized) block
+with visibility j <= i + (Nk - N) when causal (N queries, Nk keys: the
+diagonal is aligned to the last key) and the 128x128 (or ``block``-sized) block
 (i // block, j // block) kept when a block mask is given -- the definition of
 attention in [UF] "什么是注意力" with the safe softmax of [AY] "(Safe) Softmax".
 A row with no visible key gives O_i = 0 and lse_i = -inf.
@@ -20,8 +21,9 @@ import math
 
 
 def attention_brute(q, k, v, scale, causal=False, block_mask=None, block=128):
-    """q, k, v: nested lists (or arrays) [B][H][N][d].  Returns (O, lse) as lists."""
+    """q: nested lists [B][H][N][d]; k, v: [B][H][Nk][d].  Returns (O, lse) as lists."""
     B, H, N = len(q), len(q[0]), len(q[0][0])
+    Nk = len(k[0][0])
     out_o, out_l = [], []
     for b in range(B):
         ob, lb = [], []
@@ -29,8 +31,8 @@ def attention_brute(q, k, v, scale, causal=False, block_mask=None, block=128):
             oh, lh = [], []
             for i in range(N):
                 keys = []
-                for j in range(N):
-                    if causal and j > i:
+                for j in range(Nk):
+                    if causal and j - (Nk - N) > i:  # diagonal aligned to the last key
                         continue
                     if block_mask is not None and not block_mask[b][h][i // block][j // block]:
                         continue

@@ -385,3 +385,66 @@ def test_planted_mistakes_are_caught(kind, monkeypatch):
         except AssertionError:
             failed += 1
     assert failed > 0, f"no pin caught the planted mistake {kind!r}"
+
+
+# ------------------------------------------ different query / key lengths ---
+
+def _inputs_qk(B, H, Nq, Nk, d, seed, std=1.0):
+    r = _rng(seed)
+    q = _bf16(r.normal(size=(B, H, Nq, d)) * std)
+    k = _bf16(r.normal(size=(B, H, Nk, d)) * std)
+    v = _bf16(r.normal(size=(B, H, Nk, d)))
+    return q, k, v
+
+
+def _mask_qk(B, H, Nq, Nk, block, p, seed):
+    r = _rng(seed)
+    m = r.random((H, -(-Nq // block), -(-Nk // block))) < p
+    return np.broadcast_to(m[None], (B, H) + m.shape[1:]).astype(np.uint8)
+
+
+@pytest.mark.parametrize("nq,nk", [(1, 5), (3, 8), (8, 3), (6, 6), (2, 7)])
+@pytest.mark.parametrize("mode", MODES)
+def test_qk_lengths_brute_force(nq, nk, mode):
+    B, H, d, block = 1, 2, 3, 2
+    q, k, v = _inputs_qk(B, H, nq, nk, d, nq * 10 + nk, std=1.5)
+    causal = mode in ("causal", "sparse_causal")
+    mask = _mask_qk(B, H, nq, nk, block, 0.6, nq + nk) if mode.startswith("sparse") else None
+    o, lse = oracle.attention_ref(q, k, v, 0.8, causal=causal, block_mask=mask, block=block)
+    ob, lb = oracle.attention_brute(q.tolist(), k.tolist(), v.tolist(), 0.8, causal=causal,
+                                    block_mask=None if mask is None else mask.tolist(), block=block)
+    np.testing.assert_allclose(o, np.array(ob), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, np.array(lb), rtol=1e-12, atol=1e-13)
+    o2, l2 = oracle.attention_tiled_online(q, k, v, 0.8, causal=causal, block_mask=mask, block=block,
+                                           bm=3, bn=2)
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l2, lse, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("nq,nk", [(5, 40), (40, 40), (33, 17)])
+def test_qk_causal_matches_lower_right_sdpa(nq, nk):
+    """PyTorch's lower-right causal bias is the same bottom-right alignment."""
+    from torch.nn.attention.bias import causal_lower_right
+
+    B, H, d = 2, 2, 8
+    q, k, v = _inputs_qk(B, H, nq, nk, d, 31)
+    o, lse = oracle.attention_ref(q, k, v, 0.4, causal=True)
+    if nq > nk:
+        # the first nq - nk rows see no key at all
+        assert np.all(lse[:, :, : nq - nk] == -math.inf) and not o[:, :, : nq - nk].any()
+        rows = slice(nq - nk, nq)
+    else:
+        rows = slice(0, nq)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v),
+        attn_mask=causal_lower_right(nq, nk), scale=0.4).numpy()
+    np.testing.assert_allclose(o[:, :, rows], ref[:, :, rows], rtol=1e-11, atol=1e-12)
+
+
+def test_decode_row_sees_every_key():
+    B, H, nk, d = 1, 3, 50, 4
+    q, k, v = _inputs_qk(B, H, 1, nk, d, 41)
+    oc, lc = oracle.attention_ref(q, k, v, 0.6, causal=True)
+    of, lf = oracle.attention_ref(q, k, v, 0.6, causal=False)
+    np.testing.assert_array_equal(oc, of)
+    np.testing.assert_array_equal(lc, lf)
