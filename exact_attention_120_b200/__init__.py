@@ -10,6 +10,8 @@ Functions with the C names take raw device addresses:
 * ``fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask)``
 * ``fa_fwd_stream(..., stream)``
 * ``fa_fwd_qk(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, stream)``
+* ``fa_fwd_splitkv(..., num_splits, workspace, workspace_bytes, stream)`` with
+  ``fa_fwd_splitkv_workspace_bytes`` and ``fa_fwd_splitkv_heuristic``
 * ``fa_device_status(stream)``, ``fa_status_string(status)``
 
 and ``attention_forward(q, k, v, ...)`` is the tensor-level convenience that
@@ -24,7 +26,8 @@ import os
 
 __all__ = [
     "FaError", "library_path", "load_library", "fa_fwd", "fa_fwd_stream", "fa_fwd_qk",
-    "fa_device_status",
+    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_heuristic",
+    "attention_forward_splitkv", "fa_device_status",
     "fa_status_string", "fa_launches_per_call", "attention_forward", "FA_OK",
     "FA_ERR_INVALID_ARGUMENT", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT",
     "MASK_BLOCK",
@@ -50,6 +53,12 @@ _SIGNATURES = {
     "fa_fwd_qk": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
                   + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                           ctypes.c_void_p]),
+    "fa_fwd_splitkv": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
+                       + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                               ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
+                                               ctypes.c_void_p]),
+    "fa_fwd_splitkv_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 6),
+    "fa_fwd_splitkv_heuristic": (ctypes.c_int, [ctypes.c_int] * 4),
     "fa_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_cuda_error": (ctypes.c_int, []),
@@ -106,6 +115,21 @@ def fa_fwd_qk(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, strea
     """C ``fa_fwd_qk`` (Nq query rows, Nk keys) on raw device addresses."""
     return load_library().fa_fwd_qk(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask,
                                     stream)
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, num_splits,
+                   workspace, workspace_bytes, stream) -> int:
+    """C ``fa_fwd_splitkv`` on raw device addresses."""
+    return load_library().fa_fwd_splitkv(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal,
+                                         block_mask, num_splits, workspace, workspace_bytes, stream)
+
+
+def fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits) -> int:
+    return load_library().fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits)
+
+
+def fa_fwd_splitkv_heuristic(B, H, Nq, Nk) -> int:
+    return load_library().fa_fwd_splitkv_heuristic(B, H, Nq, Nk)
 
 
 def fa_device_status(stream=None) -> int:
@@ -166,4 +190,41 @@ def attention_forward(q, k, v, causal=False, block_mask=None, scale=None, out=No
                            B, H, Nq, Nk, d, float(scale), int(bool(causal)), mask_ptr, stream)
     if st != FA_OK:
         raise FaError(st, "fa_fwd")
+    return out, lse
+
+
+def attention_forward_splitkv(q, k, v, causal=False, block_mask=None, scale=None, num_splits=None,
+                              workspace=None, out=None, lse=None, stream=None):
+    """attention_forward with the keys cut into slices (fa_fwd_splitkv).
+
+    num_splits: None picks fa_fwd_splitkv_heuristic.  workspace: a CUDA uint8
+    tensor of at least fa_fwd_splitkv_workspace_bytes(...) bytes, or None to
+    allocate one with torch.  Returns (o, lse).
+    """
+    import torch
+
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if num_splits is None:
+        num_splits = fa_fwd_splitkv_heuristic(B, H, Nq, Nk)
+    need = fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    mask_ptr = None if block_mask is None else block_mask.data_ptr()
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    ws_ptr = None if workspace is None else workspace.data_ptr()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        st = fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                            B, H, Nq, Nk, d, float(scale), int(bool(causal)), mask_ptr, num_splits,
+                            ws_ptr, ws_bytes, stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_splitkv")
     return out, lse

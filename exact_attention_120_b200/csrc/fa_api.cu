@@ -15,6 +15,7 @@
 
 #include "fa.h"
 #include "fa_testing.h"
+#include "fa_combine.cuh"
 #include "fa_fwd_kernel.cuh"
 
 namespace {
@@ -120,10 +121,19 @@ int encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
   return FA_OK;
 }
 
+constexpr int kMaxSplits = 256;
+
+// Bytes of the split-key workspace: fp32 partial O [splits][rows][d] followed
+// by fp32 partial lse [splits][rows].
+size_t splitkv_workspace_bytes(size_t rows, int d, int splits) {
+  return (size_t)splits * rows * ((size_t)d + 1) * sizeof(float);
+}
+
 // Validation, descriptors and launch shared by the entry points.
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
-               void* cuda_stream, unsigned long long timeout_ns, int starve_producer) {
+               void* cuda_stream, unsigned long long timeout_ns, int starve_producer,
+               int num_splits = 1, void* workspace = nullptr, size_t workspace_bytes = 0) {
   // ---- arguments (nothing is launched on error)
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
   if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARGUMENT;
@@ -140,13 +150,25 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
       (long long)Nk * d * 2 >= (1ll << 40))
     return FA_ERR_UNSUPPORTED;  // 32-bit work indices and TMA stride limits
   if (o == q || o == k || o == v) return FA_ERR_INVALID_ARGUMENT;
+  if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARGUMENT;
+  // Slices of kt_per_split key tiles; the last one is never empty.
+  const int kt_per_split = (int)((nkt + num_splits - 1) / num_splits);
+  const int splits = (int)((nkt + kt_per_split - 1) / kt_per_split);
+  if (bh * npairs * splits > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)bh * Nq;
+  if (splits > 1) {
+    if (!workspace || !aligned(workspace, 16) ||
+        workspace_bytes < splitkv_workspace_bytes(rows, d, splits))
+      return FA_ERR_INVALID_ARGUMENT;
+  }
 
   DeviceState* st = nullptr;
   int rc = get_device_state(&st);
   if (rc != FA_OK) return rc;
   if (!is_device_pointer(q) || !is_device_pointer(k) || !is_device_pointer(v) ||
       !is_device_pointer(o) || !is_device_pointer(lse) ||
-      (block_mask && !is_device_pointer(block_mask)))
+      (block_mask && !is_device_pointer(block_mask)) ||
+      (splits > 1 && !is_device_pointer(workspace)))
     return FA_ERR_INVALID_ARGUMENT;
   if ((rc = get_encoder()) != FA_OK) return rc;
 
@@ -166,7 +188,13 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.causal_off = Nk - Nq;
   p.npairs = (int)npairs;
   p.bh = (int)bh;
-  p.items = (int)(bh * npairs);
+  p.items = (int)(bh * npairs * splits);
+  p.splits = splits;
+  p.kt_per_split = kt_per_split;
+  if (splits > 1) {
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = p.part_o + (size_t)splits * rows * d;
+  }
   p.causal = causal;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   p.timeout_ns = timeout_ns;
@@ -182,6 +210,19 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     fa::fa_fwd_kernel<128><<<grid, fa::kThreads, fa::Cfg<128>::kSmemBytes, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
+  if (splits > 1) {  // merge the slices (concatenated-softmax rule)
+    const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+    if (d == 64)
+      fa::fa_combine_kernel<64><<<blocks, 256, 0, stream>>>(p.part_o, p.part_lse,
+                                                           static_cast<__nv_bfloat16*>(o), lse,
+                                                           (long long)rows, splits);
+    else
+      fa::fa_combine_kernel<128><<<blocks, 256, 0, stream>>>(p.part_o, p.part_lse,
+                                                            static_cast<__nv_bfloat16*>(o), lse,
+                                                            (long long)rows, splits);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   return FA_OK;
 }
 
@@ -201,6 +242,34 @@ int fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, 
               void* cuda_stream) {
   return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
                     kWaitTimeoutNs, 0);
+}
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || num_splits < 1 || num_splits > kMaxSplits) return 0;
+  const long long nkt = (Nk + fa::kBN - 1) / fa::kBN;
+  const long long per = (nkt + num_splits - 1) / num_splits;
+  const int splits = (int)((nkt + per - 1) / per);
+  return splits > 1 ? splitkv_workspace_bytes((size_t)B * H * Nq, d, splits) : 0;
+}
+
+int fa_fwd_splitkv_heuristic(int B, int H, int Nq, int Nk) {
+  DeviceState* st = nullptr;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || get_device_state(&st) != FA_OK) return 1;
+  const long long units = (long long)B * H * (((Nq + fa::kBM - 1) / fa::kBM + 1) / 2);
+  const long long nkt = (Nk + fa::kBN - 1) / fa::kBN;
+  if (units >= st->num_sms || nkt < 4) return 1;
+  // About two waves of units, each slice at least two key tiles long.
+  long long splits = (2 * st->num_sms + units - 1) / units;
+  if (splits > nkt / 2) splits = nkt / 2;
+  if (splits > kMaxSplits) splits = kMaxSplits;
+  return splits < 1 ? 1 : (int)splits;
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
+                   int num_splits, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
+                    kWaitTimeoutNs, 0, num_splits, workspace, workspace_bytes);
 }
 
 int fa_testing_fwd_starved(const void* q, const void* k, const void* v, void* o, float* lse, int B,

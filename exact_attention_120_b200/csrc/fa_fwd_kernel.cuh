@@ -83,6 +83,14 @@ struct KernelParams {
   // nothing, so the first barrier wait of the MMA issuer can never complete and
   // must end through its time limit.  Always 0 on the production entry points.
   int starve_producer;
+  // Split key ranges (flash-decoding style): a work unit covers key tiles
+  // [split * kt_per_split, (split + 1) * kt_per_split).  With splits > 1 the
+  // epilogue writes the unit's normalised fp32 partial O and its partial lse to
+  // the caller's workspace instead of O and lse; fa_combine_kernel merges them.
+  int splits;
+  int kt_per_split;
+  float* part_o;    // [splits][B*H*Nq][D]
+  float* part_lse;  // [splits][B*H*Nq]
 };
 
 template <int D>
@@ -160,7 +168,10 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo,
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-__device__ __forceinline__ void decode_item(const KernelParams& p, int w, int& bh, int& pair) {
+__device__ __forceinline__ void decode_item(const KernelParams& p, int w, int& bh, int& pair,
+                                            int& split) {
+  split = w % p.splits;  // the slices of one unit run side by side
+  w /= p.splits;
   if (p.causal) {  // longest rows first, all heads interleaved
     pair = p.npairs - 1 - w / p.bh;
     bh = w % p.bh;
@@ -183,11 +194,12 @@ __device__ __forceinline__ int key_tile_end(const KernelParams& p, int qt) {
   return last < 0 ? 0 : min(p.nkt, last / kBN + 1);
 }
 
-// Bit l set <=> key tile j0 + l is visible to query tile qt (whole warp calls).
+// Bit l set <=> key tile j0 + l, which must lie in [jlo, jhi), is visible to
+// query tile qt (whole warp calls).
 __device__ __forceinline__ uint32_t keep_bits(const KernelParams& p, int bh, int qt, int j0,
-                                              int lane) {
+                                              int lane, int jlo, int jhi) {
   const int j = j0 + lane;
-  bool k = (qt < p.nqt) && (j < p.nkt);
+  bool k = (qt < p.nqt) && (j >= jlo) && (j < jhi);
   if (k && p.causal) k = j * kBN <= causal_last_key(p, qt);
   if (k && p.mask != nullptr) k = p.mask[((size_t)bh * p.nqt + qt) * p.nkt + j] != 0;
   return __ballot_sync(0xffffffffu, k);
@@ -411,10 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     uint32_t nq = 0;       // Q loads issued
     bool ok = true;
     for (int w = blockIdx.x; w < p.items && ok && !p.starve_producer; w += gridDim.x) {
-      int bh, pair;
-      decode_item(p, w, bh, pair);
+      int bh, pair, split;
+      decode_item(p, w, bh, pair, split);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
       const int nvalid = (qt1 < p.nqt) ? 2 : 1;
+      const int jb = split * p.kt_per_split, je = min(p.nkt, jb + p.kt_per_split);
       ok = wait_warp(bQEmpty, (nq & 1u) ^ 1u, abort_flag, p);
       if (ok && ptx::elect_one()) {
         ptx::mbar_arrive_expect_tx(bQFull, nvalid * C::kTileBytes);
@@ -424,9 +437,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
                              (qt0 + q) * kBM, bh);
       }
       ++nq;
-      const int jend = key_tile_end(p, qt0 + nvalid - 1);
-      for (int j0 = 0; j0 < jend && ok; j0 += 32) {
-        uint32_t u = keep_bits(p, bh, qt0, j0, lane) | keep_bits(p, bh, qt1, j0, lane);
+      const int jend = min(je, key_tile_end(p, qt0 + nvalid - 1));
+      for (int j0 = jb & ~31; j0 < jend && ok; j0 += 32) {
+        uint32_t u = keep_bits(p, bh, qt0, j0, lane, jb, je) | keep_bits(p, bh, qt1, j0, lane, jb, je);
         while (u != 0 && ok) {
           const int j = j0 + __ffs(u) - 1;
           u &= u - 1;
@@ -463,20 +476,21 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     bool ok = true;
     const MmaCtx<D> ctx{tmem, sQ, sRing, abort_flag};
     for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
-      int bh, pair;
-      decode_item(p, w, bh, pair);
+      int bh, pair, split;
+      decode_item(p, w, bh, pair, split);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
       const bool valid1 = qt1 < p.nqt;
+      const int jb = split * p.kt_per_split, je = min(p.nkt, jb + p.kt_per_split);
       slot0.begin_unit(true);
       slot1.begin_unit(valid1);
       int64_t prev_v = -1;
       ok = wait_warp(bQFull, nq & 1u, abort_flag, p);
       ptx::tc_fence_after();
       ++nq;
-      const int jend = key_tile_end(p, valid1 ? qt1 : qt0);
-      for (int j0 = 0; j0 < jend && ok; j0 += 32) {
-        const uint32_t k0 = keep_bits(p, bh, qt0, j0, lane);
-        const uint32_t k1 = keep_bits(p, bh, qt1, j0, lane);
+      const int jend = min(je, key_tile_end(p, valid1 ? qt1 : qt0));
+      for (int j0 = jb & ~31; j0 < jend && ok; j0 += 32) {
+        const uint32_t k0 = keep_bits(p, bh, qt0, j0, lane, jb, je);
+        const uint32_t k1 = keep_bits(p, bh, qt1, j0, lane, jb, je);
         uint32_t u = k0 | k1;
         while (u != 0 && ok) {
           const int l = __ffs(u) - 1;
@@ -545,17 +559,18 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     uint32_t swait = 0, owait = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
-      int bh, pair;
-      decode_item(p, w, bh, pair);
+      int bh, pair, split;
+      decode_item(p, w, bh, pair, split);
       const int qt = 2 * pair + q;
+      const int jb = split * p.kt_per_split, je = min(p.nkt, jb + p.kt_per_split);
       if (qt >= p.nqt) continue;
       const int row = qt * kBM + row_in_tile;  // query row within the head
       float m_ref = -INFINITY;  // reference max, in units of c * score
       float l = 0.f;            // sum of bf16-rounded 2^(c s - m_ref)
       int n = 0;                // tiles processed
-      const int jend = key_tile_end(p, qt);
-      for (int j0 = 0; j0 < jend && ok; j0 += 32) {
-        uint32_t kb = keep_bits(p, bh, qt, j0, lane);
+      const int jend = min(je, key_tile_end(p, qt));
+      for (int j0 = jb & ~31; j0 < jend && ok; j0 += 32) {
+        uint32_t kb = keep_bits(p, bh, qt, j0, lane, jb, je);
         while (kb != 0 && ok) {
           const int j = j0 + __ffs(kb) - 1;
           kb &= kb - 1;
@@ -677,6 +692,30 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       const bool seen = m_ref != -INFINITY && l > 0.f;
       const float inv = seen ? 1.f / l : 0.f;
       const bool in_range = row < p.Nq;
+      if (p.splits > 1) {
+        // Partial result of this key slice: normalised O (fp32) and its lse.
+        const size_t prow = (size_t)split * p.bh * p.Nq + (size_t)bh * p.Nq + (in_range ? row : 0);
+        float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t t[32];
+          if (n > 0) {
+            ptx::tmem_ld32(tO + 32 * c, t);
+            ptx::tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) t[e] = 0u;
+          }
+          if (in_range) {
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4)
+              dst[c * 8 + v4] = make_float4(__uint_as_float(t[4 * v4]) * inv, __uint_as_float(t[4 * v4 + 1]) * inv,
+                                            __uint_as_float(t[4 * v4 + 2]) * inv, __uint_as_float(t[4 * v4 + 3]) * inv);
+          }
+        }
+        if (in_range)
+          p.part_lse[prow] = seen ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      } else {
       uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -698,11 +737,12 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
             orow[c * 4 + v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
         }
       }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(bOEmpty(q));
       if (in_range)
         p.lse[(size_t)bh * p.Nq + row] =
             seen ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bOEmpty(q));
     }
   }
 

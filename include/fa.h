@@ -46,6 +46,7 @@
 #ifndef FA_B200_FA_H_
 #define FA_B200_FA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -101,6 +102,38 @@ FA_API int fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float
                      const uint8_t* block_mask, void* cuda_stream);
 
 /*
+ * Split-key ("flash-decoding") forward for problems with fewer work units than
+ * SMs, such as decoding against a long key/value cache.  The keys are cut into
+ * `num_splits` slices of whole 128-key tiles (at most 256; slices that would be
+ * empty are dropped).  Each work unit computes one slice's normalised partial
+ * output and logsumexp into `workspace`.  A second kernel merges the slices
+ * with the concatenated-softmax rule ("理解 Flash Attention", section
+ * "瓦片注意力计算") into o and lse.  Arguments and meaning are those of
+ * fa_fwd_qk.  The results equal fa_fwd_qk's up to floating-point rounding
+ * (they are not bitwise identical).
+ * workspace: device memory, 16-byte aligned, at least
+ *   fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits) bytes, owned by
+ *   the caller and overwritten by the call.  It may be NULL when that size is 0
+ *   (a single slice).
+ * Calls that share one workspace must not overlap on the GPU.  Two launches are
+ * enqueued on `cuda_stream` when there is more than one slice.
+ */
+FA_API int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int H, int Nq, int Nk, int d, float scale, int causal,
+                          const uint8_t* block_mask, int num_splits, void* workspace,
+                          size_t workspace_bytes, void* cuda_stream);
+
+/* Workspace bytes fa_fwd_splitkv needs (0 when it uses a single slice). */
+FA_API size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits);
+
+/*
+ * A slice count that keeps all SMs of the current device busy: 1 when the
+ * problem already has at least one work unit per SM, otherwise about two
+ * waves of units, each slice at least two key tiles long.
+ */
+FA_API int fa_fwd_splitkv_heuristic(int B, int H, int Nq, int Nk);
+
+/*
  * Reads and clears the device-side status word of the current device after
  * synchronising `cuda_stream`.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT (a
  * kernel's wait on one of its own barriers exceeded the time limit; the
@@ -115,7 +148,7 @@ FA_API const char* fa_status_string(int status);
 /* The cudaError_t value behind the last FA_ERR_CUDA on this host thread. */
 FA_API int fa_last_cuda_error(void);
 
-/* Number of kernel launches one fa_fwd call makes (constant: 1). */
+/* Number of kernel launches one fa_fwd / fa_fwd_qk call makes (constant: 1). */
 FA_API int fa_launches_per_call(void);
 
 #ifdef __cplusplus

@@ -67,3 +67,12 @@ def test_argument_errors_before_any_cuda_call(lib):
     assert call(q=p + 8) == fa.FA_ERR_INVALID_ARGUMENT  # not 16-byte aligned
     assert call(o=p) == fa.FA_ERR_INVALID_ARGUMENT      # o aliases q
     assert call(B=1 << 16, H=1 << 16) == fa.FA_ERR_UNSUPPORTED  # B*H beyond 32 bits
+
+
+def test_splitkv_workspace_size(lib):
+    # [splits][rows][d] fp32 partial outputs + [splits][rows] fp32 lse
+    assert fa.fa_fwd_splitkv_workspace_bytes(2, 4, 1, 16384, 128, 8) == 8 * 8 * 129 * 4
+    # 3 key tiles in at most 3 slices, whatever is asked
+    assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 10, 300, 64, 100) == 3 * 10 * 65 * 4
+    assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 10, 300, 64, 1) == 0
+    assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 10, 300, 64, 0) == 0
