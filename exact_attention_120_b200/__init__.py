@@ -58,6 +58,9 @@ _SIGNATURES = {
                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                                                ctypes.c_void_p]),
     "fa_fwd_splitkv_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 6),
+    "fa_fwd_splitkv_noalloc": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
+                               + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                                       ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_splitkv_heuristic": (ctypes.c_int, [ctypes.c_int] * 4),
     "fa_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),

@@ -123,6 +123,21 @@ int encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
 
 constexpr int kMaxSplits = 256;
 
+// Workspace of fa_fwd_splitkv_noalloc: a fixed array in the module's device
+// memory, so that entry point never allocates.  Every device that loads the
+// library holds it until the process exits; all calls on a device share it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch per device.  In host code the array's
+// name only stands in for the symbol; the address comes from
+// cudaGetSymbolAddress, taken once per device with that device current.
+struct NoallocState {
+  std::once_flag once;
+  int status = FA_ERR_CUDA;
+  void* scratch = nullptr;
+};
+NoallocState g_noalloc[kMaxDevices];
+
 // Bytes of the split-key workspace: fp32 partial O [splits][rows][d] followed
 // by fp32 partial lse [splits][rows].
 size_t splitkv_workspace_bytes(size_t rows, int d, int splits) {
@@ -270,6 +285,34 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
                    int num_splits, void* workspace, size_t workspace_bytes, void* cuda_stream) {
   return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
                     kWaitTimeoutNs, 0, num_splits, workspace, workspace_bytes);
+}
+
+int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                           int H, int Nq, int Nk, int d, float scale, int causal,
+                           const uint8_t* block_mask, int num_splits, void* cuda_stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  NoallocState& ns = g_noalloc[dev];
+  std::call_once(ns.once, [&] {  // first call on this device: find the array
+    void* ptr = nullptr;
+    const cudaError_t r = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (r != cudaSuccess) {
+      t_last_cuda_error = static_cast<int>(r);
+      ns.status = FA_ERR_CUDA;
+      return;
+    }
+    ns.scratch = ptr;
+    ns.status = FA_OK;
+  });
+  if (ns.status != FA_OK) return ns.status;
+  const size_t need = fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits);
+  if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  // The split kernel writes every partial it later reads (empty slices
+  // included), so nothing in the array has to start at zero.
+  return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
+                    kWaitTimeoutNs, 0, num_splits, need > 0 ? ns.scratch : nullptr, need);
 }
 
 int fa_testing_fwd_starved(const void* q, const void* k, const void* v, void* o, float* lse, int B,

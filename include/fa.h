@@ -126,6 +126,40 @@ FA_API int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, 
 /* Workspace bytes fa_fwd_splitkv needs (0 when it uses a single slice). */
 FA_API size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits);
 
+/* Size of the fixed device array behind fa_fwd_splitkv_noalloc (16 MiB). */
+#define FA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * fa_fwd_splitkv without a caller workspace, for callers that cannot allocate
+ * device memory at call time.  Examples: plugin code run by a host framework
+ * that owns every allocation; code on a latency-critical path that may not pay
+ * for cudaMalloc; code that runs while allocation is forbidden.  The partial
+ * results live in one fixed array of FA_NOALLOC_SCRATCH_BYTES in the library's
+ * device memory.  Every GPU that loads the library holds it until the process
+ * exits.  The call itself allocates nothing: it makes no cudaMalloc or
+ * cudaFree call, and no call to any allocating library.
+ *
+ * Arguments and results are those of fa_fwd_splitkv (num_splits >= 1), minus
+ * the workspace.  A problem whose workspace would exceed the array
+ * (fa_fwd_splitkv_workspace_bytes(...) > FA_NOALLOC_SCRATCH_BYTES) is rejected
+ * with FA_ERR_UNSUPPORTED before anything is launched.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, once per device, with that device current).  Make that
+ * first call before capturing any stream.
+ *
+ * All calls on a device share the one array, and it keeps the last call's
+ * contents.  Calls whose kernels overlap on the GPU (on different streams,
+ * without ordering between them) race on it and corrupt each other's results:
+ * serialise them.  No part of the array needs to start at zero.
+ *
+ * The pages have no counterpart to this entry point: it is a packaging of
+ * fa_fwd_splitkv for callers without an allocator.
+ */
+FA_API int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                                  const uint8_t* block_mask, int num_splits, void* cuda_stream);
+
 /*
  * A slice count that keeps all SMs of the current device busy: 1 when the
  * problem already has at least one work unit per SM, otherwise about two
