@@ -23,6 +23,7 @@ Modules:
                         and its logsumexp in float64 (NumPy), plus the one-pass
                         tiled algorithm written in the pages' order.
 * ``brute``          -- an independent pure-Python version for tiny shapes.
+* ``backward``       -- dQ, dK, dV by the chain rule through the definition.
 
 Every function here is pinned by ``tests/test_oracle.py`` to closed forms,
 invariants and the pages' worked example; see that file's header.
@@ -36,3 +37,4 @@ from .attention import (  # noqa: F401
     attention_tiled_online,
 )
 from .brute import attention_brute  # noqa: F401
+from .backward import attention_bwd_ref, softmax_delta  # noqa: F401
