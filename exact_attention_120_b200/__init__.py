@@ -12,6 +12,8 @@ Functions with the C names take raw device addresses:
 * ``fa_fwd_qk(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, stream)``
 * ``fa_fwd_splitkv(..., num_splits, workspace, workspace_bytes, stream)`` with
   ``fa_fwd_splitkv_workspace_bytes`` and ``fa_fwd_splitkv_heuristic``
+* ``fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, causal,
+  block_mask, workspace, workspace_bytes, stream)`` and ``fa_bwd_workspace_bytes``
 * ``fa_device_status(stream)``, ``fa_status_string(status)``
 
 and ``attention_forward(q, k, v, ...)`` is the tensor-level convenience that
@@ -27,7 +29,8 @@ import os
 __all__ = [
     "FaError", "library_path", "load_library", "fa_fwd", "fa_fwd_stream", "fa_fwd_qk",
     "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_heuristic",
-    "attention_forward_splitkv", "fa_device_status",
+    "attention_forward_splitkv", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward",
+    "fa_device_status",
     "fa_status_string", "fa_launches_per_call", "attention_forward", "FA_OK",
     "FA_ERR_INVALID_ARGUMENT", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT",
     "MASK_BLOCK",
@@ -62,6 +65,10 @@ _SIGNATURES = {
                                + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                                        ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_splitkv_heuristic": (ctypes.c_int, [ctypes.c_int] * 4),
+    "fa_bwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
+               + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                  ctypes.c_void_p]),
+    "fa_bwd_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 3),
     "fa_device_status": (ctypes.c_int, [ctypes.c_void_p]),
     "fa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fa_last_cuda_error": (ctypes.c_int, []),
@@ -231,3 +238,41 @@ def attention_forward_splitkv(q, k, v, causal=False, block_mask=None, scale=None
     if st != FA_OK:
         raise FaError(st, "fa_fwd_splitkv")
     return out, lse
+
+
+def fa_bwd_workspace_bytes(B, H, Nq) -> int:
+    return load_library().fa_bwd_workspace_bytes(B, H, Nq)
+
+
+def attention_backward(q, k, v, o, lse, dout, causal=False, block_mask=None, scale=None,
+                       workspace=None, stream=None):
+    """dq, dk, dv of attention_forward through the C ABI (fa_bwd).
+
+    q, o, dout: CUDA bf16 [B, H, Nq, d]; k, v: [B, H, Nk, d]; lse: fp32
+    [B, H, Nq] from the forward; causal / block_mask / scale as in the forward.
+    """
+    import torch
+
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v, o, dout must be contiguous CUDA bfloat16 tensors")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    need = fa_bwd_workspace_bytes(B, H, Nq)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    mask_ptr = None if block_mask is None else block_mask.data_ptr()
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        st = load_library().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                   dv.data_ptr(), B, H, Nq, Nk, d, float(scale), int(bool(causal)),
+                                   mask_ptr, workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(), stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd")
+    return dq, dk, dv

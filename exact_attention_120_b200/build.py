@@ -21,7 +21,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 SOURCES = [os.path.join(CSRC, "fa_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_combine.cuh", "ptx.cuh")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_combine.cuh", "fa_bwd_kernel.cuh", "ptx.cuh")] + [
     os.path.join(INCLUDE, "fa.h"), os.path.join(INCLUDE, "fa_testing.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -8,6 +8,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
+#include <initializer_list>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -15,6 +17,7 @@
 
 #include "fa.h"
 #include "fa_testing.h"
+#include "fa_bwd_kernel.cuh"
 #include "fa_combine.cuh"
 #include "fa_fwd_kernel.cuh"
 
@@ -60,6 +63,18 @@ int setup_device(int dev, DeviceState& st) {
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaFuncSetAttribute(fa::fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            fa::Cfg<128>::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           fa::BwdCfg<64>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::BwdCfg<128>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::BwdCfg<64>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::BwdCfg<128>::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e);
   void* sym = nullptr;
   e = cudaGetSymbolAddress(&sym, g_fa_status);
@@ -313,6 +328,85 @@ int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o,
   // included), so nothing in the array has to start at zero.
   return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
                     kWaitTimeoutNs, 0, num_splits, need > 0 ? ns.scratch : nullptr, need);
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int Nq) {
+  if (B < 1 || H < 1 || Nq < 1) return 0;
+  return ((size_t)B * H * Nq * sizeof(float) + 15) / 16 * 16;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,
+           float scale, int causal, const uint8_t* block_mask, void* workspace,
+           size_t workspace_bytes, void* cuda_stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return FA_ERR_INVALID_ARGUMENT;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARGUMENT;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARGUMENT;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  for (const void* ptr : std::initializer_list<const void*>{q, k, v, o, dout, dq, dk, dv, workspace})
+    if (!aligned(ptr, 16)) return FA_ERR_INVALID_ARGUMENT;
+  if (!aligned(lse, 4)) return FA_ERR_INVALID_ARGUMENT;
+  const long long bh = (long long)B * H;
+  const long long nqt = (Nq + fa::kBM - 1) / fa::kBM;
+  const long long nkt = (Nk + fa::kBN - 1) / fa::kBN;
+  if (bh * nqt > INT32_MAX || bh * nkt > INT32_MAX || (long long)Nq * d * 2 >= (1ll << 40) ||
+      (long long)Nk * d * 2 >= (1ll << 40))
+    return FA_ERR_UNSUPPORTED;
+  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, Nq)) return FA_ERR_INVALID_ARGUMENT;
+  for (const void* out : std::initializer_list<const void*>{dq, dk, dv})
+    if (out == q || out == k || out == v || out == o || out == dout) return FA_ERR_INVALID_ARGUMENT;
+  if (dq == dk || dq == dv || dk == dv) return FA_ERR_INVALID_ARGUMENT;
+
+  DeviceState* st = nullptr;
+  int rc = get_device_state(&st);
+  if (rc != FA_OK) return rc;
+  for (const void* ptr :
+       std::initializer_list<const void*>{q, k, v, o, lse, dout, dq, dk, dv, workspace})
+    if (!is_device_pointer(ptr)) return FA_ERR_INVALID_ARGUMENT;
+  if (block_mask && !is_device_pointer(block_mask)) return FA_ERR_INVALID_ARGUMENT;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+
+  fa::BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  if ((rc = encode_qkv_map(&p.tm_q, q, (int)bh, Nq, d)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_k, k, (int)bh, Nk, d)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_v, v, (int)bh, Nk, d)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_do, dout, (int)bh, Nq, d)) != FA_OK) return rc;
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.lse = lse;
+  p.delta = static_cast<float*>(workspace);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.mask = block_mask;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.nqt = (int)nqt;
+  p.nkt = (int)nkt;
+  p.causal_off = Nk - Nq;
+  p.bh = (int)bh;
+  p.causal = causal;
+  p.scale = scale;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.timeout_ns = kWaitTimeoutNs;
+  p.status = st->status_word;
+
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  const int grid_q = (int)std::min<long long>(bh * nqt, st->num_sms);
+  const int grid_k = (int)std::min<long long>(bh * nkt, st->num_sms);
+  if (d == 64) {
+    fa::fa_bwd_dq_kernel<64><<<grid_q, fa::kBwdThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(p);
+    fa::fa_bwd_dkdv_kernel<64><<<grid_k, fa::kBwdThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(p);
+  } else {
+    fa::fa_bwd_dq_kernel<128><<<grid_q, fa::kBwdThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(p);
+    fa::fa_bwd_dkdv_kernel<128><<<grid_k, fa::kBwdThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(p);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
 }
 
 int fa_testing_fwd_starved(const void* q, const void* k, const void* v, void* o, float* lse, int B,

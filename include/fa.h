@@ -168,6 +168,30 @@ FA_API int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, v
 FA_API int fa_fwd_splitkv_heuristic(int B, int H, int Nq, int Nk);
 
 /*
+ * Backward pass: dQ, dK, dV of the forward above for the upstream gradient
+ * dO.  The scores are recomputed from q, k and the forward's lse, not stored
+ * ("理解 Flash Attention", section "瓦片注意力计算"), with P = exp(S - lse),
+ *   dV = P^T dO,  dP = dO V^T,  D_i = dO_i . O_i,  dS = P o (dP - D),
+ *   dQ = scale dS K,  dK = scale dS^T Q.
+ * q, o, dout, dq: bf16 [B, H, Nq, d]; k, v, dk, dv: bf16 [B, H, Nk, d]; lse:
+ * fp32 [B, H, Nq] as written by the forward; causal, block_mask, scale and d
+ * exactly as passed to the forward (fa_fwd / fa_fwd_qk).  All device memory,
+ * 16-byte aligned (lse: 4), owned by the caller; dq, dk, dv must not alias
+ * the inputs or each other.
+ * workspace: device memory of at least fa_bwd_workspace_bytes(B, H, Nq) bytes,
+ *   16-byte aligned, overwritten (it receives D).  Calls sharing a workspace
+ *   must not overlap on the GPU.
+ * Two kernels are enqueued on `cuda_stream` (dQ with D, then dK and dV).
+ */
+FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dout, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk,
+                  int d, float scale, int causal, const uint8_t* block_mask, void* workspace,
+                  size_t workspace_bytes, void* cuda_stream);
+
+/* Workspace bytes fa_bwd needs: one fp32 per query row, rounded to 16. */
+FA_API size_t fa_bwd_workspace_bytes(int B, int H, int Nq);
+
+/*
  * Reads and clears the device-side status word of the current device after
  * synchronising `cuda_stream`.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT (a
  * kernel's wait on one of its own barriers exceeded the time limit; the
