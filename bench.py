@@ -2,6 +2,7 @@
 """Benchmark of the fused attention forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--pass fwd|bwd]
 
 One step = one fa_fwd launch over one batch of the workload (default: the
 long full-attention workload B=1, H=16, N=16384, d=128, Q/K std 3 -- the
@@ -17,6 +18,9 @@ buffers, copies included.  ``roofline`` relates the kernel to the measured
 dense-bf16 tensor peak.  ``cpu_baseline`` times the float64 CPU oracle on a
 bounded sample of the same workload.  ``--impl reference`` times that oracle
 alone as the reference arm.
+
+``--pass bwd`` times fa_bwd (dQ, dK, dV from the forward's O and lse) on the
+same workload instead, credited with 2.5x the forward's FLOPs.
 
 Multi-GPU (launched by torchrun): ranks share nothing on the data path; each
 rank runs the full workload shape on its own batch slice (weak scaling).
@@ -68,15 +72,15 @@ def load_peaks():
         return FALLBACK_PEAK_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_hash() -> str:
+def kernel_hash(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def load_traffic(workload: str):
+def load_traffic(workload: str, pass_: str = "fwd", khash: str | None = None):
     """DRAM bytes per launch from the committed ncu summary, only if it was
     taken on the current kernel sources."""
     try:
@@ -84,8 +88,8 @@ def load_traffic(workload: str):
             rec = json.load(f)
     except (OSError, ValueError):
         return None
-    entry = rec.get(workload)
-    if not entry or entry.get("kernel_hash") != kernel_hash():
+    entry = rec.get(workload if pass_ == "fwd" else f"{pass_}:{workload}")
+    if not entry or entry.get("kernel_hash") != (khash or kernel_hash()):
         return None
     return float(entry["dram_bytes_per_launch"])
 
@@ -236,6 +240,159 @@ def workload_config(w, world):
                   % (algorithmic_bytes(w.B, w.H, w.N, w.d) // 2**20)}
 
 
+def bwd_oracle_sample(w, q, k, v, mask, n_max=2048):
+    """Time the float64 gradient oracle on head (0, 0) of the workload cut to
+    its first n_max queries and keys.  Returns (credited_flops, seconds, n)."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    n = min(w.N, n_max)
+    f = lambda t: t[0:1, 0:1, :n].to(torch.float64).numpy()  # noqa: E731
+    g = torch.Generator().manual_seed(w.seed + 7)
+    do = torch.randn((1, 1, n, w.d), generator=g).to(torch.bfloat16)
+    bm = None
+    if mask is not None:
+        nb = (n + 127) // 128
+        bm = np.ascontiguousarray(mask[0:1, 0:1, :nb, :nb].numpy())
+    t0 = time.perf_counter()
+    oracle.attention_bwd_ref(f(q), f(k), f(v), f(do), w.scale, causal=w.causal, block_mask=bm)
+    t = time.perf_counter() - t0
+    flops = 2.5 * useful_flops(1, 1, n, w.d, w.causal, None if bm is None else torch.from_numpy(bm))
+    return flops, t, n
+
+
+class FwdJob:
+    """One step = one fa_fwd launch (one forward pass over the workload)."""
+
+    name = "fwd"
+    metric = METRIC
+    kernel_sources = KERNEL_SOURCES
+
+    def __init__(self, fa, torch, w, q, k, v, mask, dev, stream):
+        self.fa, self.w = fa, w
+        self.flops = useful_flops(w.B, w.H, w.N, w.d, w.causal, mask)
+        self.q, self.k, self.v, self.mask = q, k, v, mask
+        self.qd, self.kd, self.vd = q.to(dev), k.to(dev), v.to(dev)
+        self.md = None if mask is None else mask.to(dev)
+        self.od = torch.empty_like(self.qd)
+        self.ld = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        self.stream = stream
+        self.ptrs = (self.qd.data_ptr(), self.kd.data_ptr(), self.vd.data_ptr(),
+                     self.od.data_ptr(), self.ld.data_ptr())
+        self.mptr = None if self.md is None else self.md.data_ptr()
+        self.launches_per_step = fa.fa_launches_per_call()
+
+    def launch(self):
+        w, fa = self.w, self.fa
+        st = fa.fa_fwd_stream(*self.ptrs, w.B, w.H, w.N, w.d, w.scale, int(w.causal), self.mptr,
+                              self.stream.cuda_stream)
+        if st != fa.FA_OK:
+            raise fa.FaError(st, "fa_fwd_stream")
+
+    def host_buffers(self):
+        self.hin = [t.pin_memory() for t in (self.q, self.k, self.v)]
+        self.hm = None if self.mask is None else self.mask.pin_memory()
+        self.hout = [__import__("torch").empty(t.shape, dtype=t.dtype).pin_memory()
+                     for t in (self.od, self.ld)]
+        h2d = sum(t.numel() * t.element_size() for t in self.hin) + (0 if self.hm is None else self.hm.numel())
+        d2h = sum(t.numel() * t.element_size() for t in self.hout)
+        return h2d, d2h
+
+    def e2e_step(self):
+        for d, h in zip((self.qd, self.kd, self.vd), self.hin):
+            d.copy_(h, non_blocking=True)
+        if self.hm is not None:
+            self.md.copy_(self.hm, non_blocking=True)
+        w = self.w
+        self.fa.attention_forward(self.qd, self.kd, self.vd, causal=w.causal, block_mask=self.md,
+                                  scale=w.scale, out=self.od, lse=self.ld)
+        for h, d in zip(self.hout, (self.od, self.ld)):
+            h.copy_(d, non_blocking=True)
+
+    def algorithmic_bytes(self):
+        w = self.w
+        return algorithmic_bytes(w.B, w.H, w.N, w.d)
+
+    def cpu_baseline(self, args):
+        w = self.w
+        qn, kn, vn, mn = numpy_inputs(self.q, self.k, self.v, self.mask)
+        f, t, rows = oracle_sample(w, qn, kn, vn, mn, args.cpu_rows, budget_s=args.cpu_budget)
+        return {"value": f / t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{rows} query rows of {w.name} (complete rows over all N={w.N} keys, "
+                          f"head-major from row 0), {t:.1f} s of float64 NumPy/BLAS oracle"}
+
+
+class BwdJob(FwdJob):
+    """One step = one fa_bwd call (dQ kernel + dK/dV kernel) on the forward's
+    O and lse, for a seeded upstream gradient dO.  Credited FLOPs: 2.5x the
+    forward's (five products of the forward's size against its two)."""
+
+    name = "bwd"
+    metric = "fused attention bwd TFLOP/s (bf16 dQ, dK, dV; 2.5x forward FLOPs) and % of dense BF16 peak"
+    kernel_sources = ("exact_attention_120_b200/csrc/fa_bwd_kernel.cuh",
+                      "exact_attention_120_b200/csrc/ptx.cuh",
+                      "exact_attention_120_b200/csrc/fa_api.cu")
+
+    def __init__(self, fa, torch, w, q, k, v, mask, dev, stream):
+        super().__init__(fa, torch, w, q, k, v, mask, dev, stream)
+        self.flops *= 2.5
+        g = torch.Generator().manual_seed(w.seed + 7)
+        self.do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+        self.dod = self.do.to(dev)
+        super().launch()  # O and lse of the forward, the backward's inputs
+        torch.cuda.synchronize(dev)
+        self.ho_lse = None
+        self.dq, self.dk, self.dv = (torch.empty_like(t) for t in (self.qd, self.kd, self.vd))
+        self.ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.H, w.N), dtype=torch.uint8, device=dev)
+        self.bptrs = (self.qd.data_ptr(), self.kd.data_ptr(), self.vd.data_ptr(), self.od.data_ptr(),
+                      self.ld.data_ptr(), self.dod.data_ptr(), self.dq.data_ptr(), self.dk.data_ptr(),
+                      self.dv.data_ptr())
+        self.launches_per_step = 2
+
+    def launch(self):
+        w, fa = self.w, self.fa
+        st = fa.fa_bwd(*self.bptrs, w.B, w.H, w.N, w.N, w.d, w.scale, int(w.causal), self.mptr,
+                       self.ws.data_ptr(), self.ws.numel(), self.stream.cuda_stream)
+        if st != fa.FA_OK:
+            raise fa.FaError(st, "fa_bwd")
+
+    def host_buffers(self):
+        torch = __import__("torch")
+        self.hin = [t.pin_memory() for t in (self.q, self.k, self.v)]
+        self.hin += [self.od.cpu().pin_memory(), self.ld.cpu().pin_memory(), self.do.pin_memory()]
+        self.hm = None if self.mask is None else self.mask.pin_memory()
+        self.hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (self.dq, self.dk, self.dv)]
+        h2d = sum(t.numel() * t.element_size() for t in self.hin) + (0 if self.hm is None else self.hm.numel())
+        d2h = sum(t.numel() * t.element_size() for t in self.hout)
+        return h2d, d2h
+
+    def e2e_step(self):
+        devs = (self.qd, self.kd, self.vd, self.od, self.ld, self.dod)
+        for d, h in zip(devs, self.hin):
+            d.copy_(h, non_blocking=True)
+        if self.hm is not None:
+            self.md.copy_(self.hm, non_blocking=True)
+        w = self.w
+        grads = self.fa.attention_backward(self.qd, self.kd, self.vd, self.od, self.ld, self.dod,
+                                           causal=w.causal, block_mask=self.md, scale=w.scale,
+                                           workspace=self.ws)
+        for h, d in zip(self.hout, grads):
+            h.copy_(d, non_blocking=True)
+
+    def algorithmic_bytes(self):
+        # Q, K, V, O, dO read, dQ, dK, dV written (bf16), lse read (fp32).
+        w = self.w
+        return float(w.B * w.H * (16 * w.N * w.d + 4 * w.N))
+
+    def cpu_baseline(self, args):
+        f, t, n = bwd_oracle_sample(self.w, self.q, self.k, self.v, self.mask)
+        return {"value": f / t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                "sample": f"float64 gradient oracle on head (0,0) of {self.w.name} cut to its first "
+                          f"{n} queries and keys, {t:.1f} s"}
+
+
 def run_ours(args, info):
     import torch
 
@@ -251,29 +408,18 @@ def run_ours(args, info):
     w = WORKLOADS[args.workload]
     wr = dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank))
     q, k, v, mask = make_inputs(wr)
-    flops = useful_flops(w.B, w.H, w.N, w.d, w.causal, mask)
-    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    md = None if mask is None else mask.to(dev)
-    od = torch.empty_like(qd)
-    ld = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    ptrs = (qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), ld.data_ptr())
-    mptr = None if md is None else md.data_ptr()
-
-    def launch():
-        st = fa.fa_fwd_stream(*ptrs, w.B, w.H, w.N, w.d, w.scale, int(w.causal), mptr,
-                              stream.cuda_stream)
-        if st != fa.FA_OK:
-            raise fa.FaError(st, "fa_fwd_stream")
+    job = (BwdJob if args.pass_ == "bwd" else FwdJob)(fa, torch, w, q, k, v, mask, dev, stream)
+    flops = job.flops
 
     for _ in range(args.warmup):
-        launch()
+        job.launch()
     torch.cuda.synchronize(dev)
     st = fa.fa_device_status(stream.cuda_stream)
     if st != fa.FA_OK:
         raise fa.FaError(st, "device status after warm-up")
 
-    # ---- device-timed region: K launches, inputs resident in HBM
+    # ---- device-timed region: K steps, inputs resident in HBM
     sampler = ClockSampler(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sharding.barrier(dev)
@@ -281,7 +427,7 @@ def run_ours(args, info):
     sampler.start()
     e0.record(stream)
     for _ in range(args.steps):
-        launch()
+        job.launch()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     sampler.stop()
@@ -293,36 +439,19 @@ def run_ours(args, info):
     if st != fa.FA_OK:
         raise fa.FaError(st, "device status after timed region")
 
-    # ---- end to end: pinned host inputs -> device -> fa_fwd -> host outputs
-    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    hm = None if mask is None else mask.pin_memory()
-    ho = torch.empty(od.shape, dtype=od.dtype).pin_memory()
-    hl = torch.empty(ld.shape, dtype=ld.dtype).pin_memory()
-
-    def e2e_step():
-        qd.copy_(hq, non_blocking=True)
-        kd.copy_(hk, non_blocking=True)
-        vd.copy_(hv, non_blocking=True)
-        if hm is not None:
-            md.copy_(hm, non_blocking=True)
-        fa.attention_forward(qd, kd, vd, causal=w.causal, block_mask=md, scale=w.scale, out=od,
-                             lse=ld)
-        ho.copy_(od, non_blocking=True)
-        hl.copy_(ld, non_blocking=True)
-
+    # ---- end to end: pinned host inputs -> device -> public API -> host outputs
+    h2d, d2h = job.host_buffers()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(min(3, args.warmup)):
-        e2e_step()
+        job.e2e_step()
     torch.cuda.synchronize(dev)
     sharding.barrier(dev)
     e0.record(stream)
     for _ in range(e2e_steps):
-        e2e_step()
+        job.e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sharding.max_over_ranks(e0.elapsed_time(e1), dev) / e2e_steps
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (0 if hm is None else hm.numel())
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     clocks = sampler.summary()
     if info.world_size > 1:
@@ -337,34 +466,33 @@ def run_ours(args, info):
         return 0
 
     peak, peak_sus, peak_src = load_peaks()
-    achieved = flops / (ms_step * 1e-3) / 1e12  # one launch per step
+    achieved = flops / (ms_step * 1e-3) / 1e12  # one call per step
     value = info.world_size * achieved
     cpu = None
     if info.world_size == 1 and not args.no_cpu_baseline:
-        qn, kn, vn, mn = numpy_inputs(q, k, v, mask)
-        f, t, rows = oracle_sample(w, qn, kn, vn, mn, args.cpu_rows, budget_s=args.cpu_budget)
-        cpu = {"value": f / t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{rows} query rows of {w.name} (complete rows over all N={w.N} keys, "
-                         f"head-major from row 0), {t:.1f} s of float64 NumPy/BLAS oracle"}
+        cpu = job.cpu_baseline(args)
+    khash = kernel_hash(job.kernel_sources)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world_size,
+        "metric": job.metric, "value": value, "unit": UNIT, "n_gpus": info.world_size,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) draws, bf16)", "config": workload_config(w, info.world_size),
         "pct_of_dense_bf16_peak": 100.0 * achieved / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
-                     "frac": achieved / peak, "traffic": load_traffic(w.name),
+                     "frac": achieved / peak, "traffic": load_traffic(w.name, job.name, khash),
                      "peak_kind": f"{peak_src} burst dense bf16",
                      "frac_of_sustained_peak": achieved / peak_sus,
-                     "algorithmic_bytes": algorithmic_bytes(w.B, w.H, w.N, w.d),
+                     "algorithmic_bytes": job.algorithmic_bytes(),
                      "flops_per_launch": flops},
         "e2e": {"value": info.world_size * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * fa.fa_launches_per_call(),
+        "gpu_launches": args.steps * job.launches_per_step,
         "clocks": clocks,
         "cpu_baseline": cpu,
-        "kernel_hash": kernel_hash(),
+        "kernel_hash": khash,
     }
+    if job.name == "bwd":
+        line["config"]["pass"] = "backward (fa_bwd: dQ kernel then dK/dV kernel)"
     print(json.dumps(line), flush=True)
     return 0
 
@@ -376,6 +504,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="long_full", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="time the forward (default) or the backward pass")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per timed chunk")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
@@ -389,6 +519,8 @@ def main(argv=None):
         if info.world_size == 1 and args.gpus > 1:
             ap.error("--gpus N > 1 must be launched with torchrun (one process per GPU)")
     if args.impl == "reference":
+        if args.pass_ != "fwd":
+            ap.error("--impl reference times the forward oracle only")
         return run_reference(args, info)
     return run_ours(args, info)
 
