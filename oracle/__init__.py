@@ -24,6 +24,8 @@ Modules:
                         tiled algorithm written in the pages' order.
 * ``brute``          -- an independent pure-Python version for tiny shapes.
 * ``backward``       -- dQ, dK, dV by the chain rule through the definition.
+* ``varlen``         -- variable-length batches: independent sequences packed
+                        token-major without padding.
 
 Every function here is pinned by ``tests/test_oracle.py`` to closed forms,
 invariants and the pages' worked example; see that file's header.
@@ -38,3 +40,4 @@ from .attention import (  # noqa: F401
 )
 from .brute import attention_brute  # noqa: F401
 from .backward import attention_bwd_ref, softmax_delta  # noqa: F401
+from .varlen import attention_varlen_ref  # noqa: F401
