@@ -20,7 +20,9 @@ bounded sample of the same workload.  ``--impl reference`` times that oracle
 alone as the reference arm.
 
 ``--pass bwd`` times fa_bwd (dQ, dK, dV from the forward's O and lse) on the
-same workload instead, credited with 2.5x the forward's FLOPs.
+same workload instead, credited with 2.5x the forward's FLOPs.  ``--pass
+varlen`` times fa_fwd_varlen on varlen_mix (32 causal sequences of 128 to 8192
+tokens packed without padding, H=16, d=128).
 
 Multi-GPU (launched by torchrun): ranks share nothing on the data path; each
 rank runs the full workload shape on its own batch slice (weak scaling).
@@ -43,8 +45,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_attention_120_b200 import sharding  # noqa: E402
-from exact_attention_120_b200.workloads import (WORKLOADS, algorithmic_bytes, make_inputs,  # noqa: E402
-                                                useful_flops)
+from exact_attention_120_b200.workloads import (VARLEN_WORKLOADS, WORKLOADS, algorithmic_bytes,  # noqa: E402
+                                                make_inputs, make_varlen_inputs, useful_flops,
+                                                varlen_flops)
 
 METRIC = "fused attention fwd TFLOP/s (bf16, causal & full) and % of dense BF16 peak"
 UNIT = "TFLOP/s"
@@ -393,6 +396,89 @@ class BwdJob(FwdJob):
                           f"{n} queries and keys, {t:.1f} s"}
 
 
+class VarlenJob(FwdJob):
+    """One step = one fa_fwd_varlen launch over a packed batch of sequences of
+    mixed lengths (the varlen_mix workload)."""
+
+    name = "varlen"
+    metric = "fused attention fwd TFLOP/s, variable-length batch (bf16) and % of dense BF16 peak"
+
+    def __init__(self, fa, torch, w, dev, stream):
+        self.fa, self.w, self.stream = fa, w, stream
+        self.lens, q, k, v, cu_q, cu_k = make_varlen_inputs(w)
+        self.flops = varlen_flops(self.lens, self.lens, w.H, w.d, w.causal)
+        self.q, self.k, self.v, self.cu = q, k, v, cu_q
+        self.qd, self.kd, self.vd = q.to(dev), k.to(dev), v.to(dev)
+        self.cud = cu_q.to(dev)
+        self.od = torch.empty_like(self.qd)
+        self.ld = torch.empty((w.H, q.shape[0]), dtype=torch.float32, device=dev)
+        self.max_q = max(self.lens)
+        self.launches_per_step = 1
+        self.mask = None
+
+    def launch(self):
+        w, fa = self.w, self.fa
+        st = fa.fa_fwd_varlen(self.qd.data_ptr(), self.kd.data_ptr(), self.vd.data_ptr(),
+                              self.od.data_ptr(), self.ld.data_ptr(), self.cud.data_ptr(),
+                              self.cud.data_ptr(), w.B, w.H, self.qd.shape[0], self.kd.shape[0],
+                              self.max_q, w.d, w.scale, int(w.causal), self.stream.cuda_stream)
+        if st != fa.FA_OK:
+            raise fa.FaError(st, "fa_fwd_varlen")
+
+    def host_buffers(self):
+        torch = __import__("torch")
+        self.hin = [t.pin_memory() for t in (self.q, self.k, self.v, self.cu)]
+        self.hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (self.od, self.ld)]
+        h2d = sum(t.numel() * t.element_size() for t in self.hin)
+        d2h = sum(t.numel() * t.element_size() for t in self.hout)
+        return h2d, d2h
+
+    def e2e_step(self):
+        for d, h in zip((self.qd, self.kd, self.vd, self.cud), self.hin):
+            d.copy_(h, non_blocking=True)
+        w = self.w
+        self.fa.attention_forward_varlen(self.qd, self.kd, self.vd, self.cud, self.cud, self.max_q,
+                                         causal=w.causal, scale=w.scale, out=self.od, lse=self.ld)
+        for h, d in zip(self.hout, (self.od, self.ld)):
+            h.copy_(d, non_blocking=True)
+
+    def algorithmic_bytes(self):
+        w, T = self.w, self.qd.shape[0]
+        return float(w.H * (8 * T * w.d + 4 * T))
+
+    def cpu_baseline(self, args):
+        import oracle
+
+        # The oracle on whole sequences, shortest first, head 0, ~cpu_budget s.
+        order = sorted(range(len(self.lens)), key=lambda b: self.lens[b])
+        cu = self.cu.tolist()
+        f64 = lambda t: t.to(__import__("torch").float64).numpy()  # noqa: E731
+        flops, t_total, done = 0.0, 0.0, 0
+        for b in order:
+            sl = slice(cu[b], cu[b + 1])
+            qs, ks, vs = f64(self.q[sl, 0:1]), f64(self.k[sl, 0:1]), f64(self.v[sl, 0:1])
+            n = self.lens[b]
+            t0 = time.perf_counter()
+            oracle.attention_varlen_ref(qs, ks, vs, [0, n], [0, n], self.w.scale, causal=self.w.causal)
+            t_total += time.perf_counter() - t0
+            flops += varlen_flops([n], [n], 1, self.w.d, self.w.causal)
+            done += 1
+            if t_total >= args.cpu_budget:
+                break
+        return {"value": flops / t_total / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                "sample": f"float64 oracle on head 0 of the {done} shortest sequences of {self.w.name}, "
+                          f"{t_total:.1f} s"}
+
+
+def varlen_config(w, job, world):
+    return {"workload": f"{w.name}: {w.describe()}, scale 1/sqrt(d), seed {w.seed}",
+            "B": w.B, "H": w.H, "d": w.d, "causal": w.causal, "total_tokens": int(job.qd.shape[0]),
+            "max_seqlen": job.max_q, "global_batch": w.B * world,
+            "parallelism": "replicas" if world == 1 else f"dp{world} (independent batch slices)",
+            "l2": "Q, K, V, O = %d MB per step, larger than L2; no flush"
+                  % (job.algorithmic_bytes() // 2**20)}
+
+
 def run_ours(args, info):
     import torch
 
@@ -405,11 +491,16 @@ def run_ours(args, info):
     sharding.init_process_group(info, "nccl")
     fa.load_library()
 
-    w = WORKLOADS[args.workload]
-    wr = dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank))
-    q, k, v, mask = make_inputs(wr)
     stream = torch.cuda.current_stream(dev)
-    job = (BwdJob if args.pass_ == "bwd" else FwdJob)(fa, torch, w, q, k, v, mask, dev, stream)
+    if args.pass_ == "varlen":
+        w = VARLEN_WORKLOADS["varlen_mix"]
+        job = VarlenJob(fa, torch, dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank)),
+                        dev, stream)
+    else:
+        w = WORKLOADS[args.workload]
+        wr = dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank))
+        q, k, v, mask = make_inputs(wr)
+        job = (BwdJob if args.pass_ == "bwd" else FwdJob)(fa, torch, w, q, k, v, mask, dev, stream)
     flops = job.flops
 
     for _ in range(args.warmup):
@@ -476,7 +567,9 @@ def run_ours(args, info):
         "metric": job.metric, "value": value, "unit": UNIT, "n_gpus": info.world_size,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) draws, bf16)", "config": workload_config(w, info.world_size),
+        "data": "synthetic (seeded N(0,1) draws, bf16)",
+        "config": (varlen_config(w, job, info.world_size) if job.name == "varlen"
+                   else workload_config(w, info.world_size)),
         "pct_of_dense_bf16_peak": 100.0 * achieved / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": load_traffic(w.name, job.name, khash),
@@ -504,8 +597,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="long_full", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
-                    help="time the forward (default) or the backward pass")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "varlen"],
+                    help="time the forward (default), the backward pass, or the forward on the "
+                         "variable-length batch varlen_mix (--workload is then ignored)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per timed chunk")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")

@@ -30,7 +30,7 @@ __all__ = [
     "FaError", "library_path", "load_library", "fa_fwd", "fa_fwd_stream", "fa_fwd_qk",
     "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_heuristic",
     "attention_forward_splitkv", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward",
-    "fa_device_status",
+    "fa_device_status", "fa_fwd_varlen", "attention_forward_varlen",
     "fa_status_string", "fa_launches_per_call", "attention_forward", "FA_OK",
     "FA_ERR_INVALID_ARGUMENT", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT",
     "MASK_BLOCK",
@@ -65,6 +65,8 @@ _SIGNATURES = {
                                + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                                        ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_splitkv_heuristic": (ctypes.c_int, [ctypes.c_int] * 4),
+    "fa_fwd_varlen": (ctypes.c_int, [ctypes.c_void_p] * 7 + [ctypes.c_int] * 6
+                      + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
     "fa_bwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
                + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                   ctypes.c_void_p]),
@@ -240,6 +242,18 @@ def attention_forward_splitkv(q, k, v, causal=False, block_mask=None, scale=None
     return out, lse
 
 
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, causal, block_mask, workspace,
+           workspace_bytes, stream) -> int:
+    return load_library().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, causal,
+                                 block_mask, workspace, workspace_bytes, stream)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, max_seqlen_q,
+                  d, scale, causal, stream) -> int:
+    return load_library().fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q,
+                                        total_k, max_seqlen_q, d, scale, causal, stream)
+
+
 def fa_bwd_workspace_bytes(B, H, Nq) -> int:
     return load_library().fa_bwd_workspace_bytes(B, H, Nq)
 
@@ -276,3 +290,43 @@ def attention_backward(q, k, v, o, lse, dout, causal=False, block_mask=None, sca
     if st != FA_OK:
         raise FaError(st, "fa_bwd")
     return dq, dk, dv
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, causal=False,
+                             scale=None, out=None, lse=None, stream=None):
+    """O, lse of a variable-length batch through the C ABI (fa_fwd_varlen).
+
+    q: CUDA bf16 [total_q, H, d]; k, v: [total_k, H, d] (packed tokens);
+    cu_seqlens_q / cu_seqlens_k: CUDA int32 [B + 1] offsets; max_seqlen_q:
+    the longest query sequence.  Returns O [total_q, H, d] and lse
+    [H, total_q] (fp32).
+    """
+    import torch
+
+    Tq, H, d = q.shape
+    Tk = k.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA bfloat16 tensors")
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("cu_seqlens must be contiguous CUDA int32 tensors")
+    B = cu_seqlens_q.numel() - 1
+    if cu_seqlens_k.numel() != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        st = load_library().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                          lse.data_ptr(), cu_seqlens_q.data_ptr(),
+                                          cu_seqlens_k.data_ptr(), B, H, Tq, Tk, int(max_seqlen_q), d,
+                                          float(scale), int(bool(causal)), stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_varlen")
+    return out, lse

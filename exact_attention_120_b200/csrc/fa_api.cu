@@ -63,6 +63,12 @@ int setup_device(int dev, DeviceState& st) {
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaFuncSetAttribute(fa::fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            fa::Cfg<128>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa::fa_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::Cfg<64>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa::fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::Cfg<128>::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            fa::BwdCfg<64>::kSmemBytes);
@@ -124,6 +130,24 @@ int encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
   const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    t_last_cuda_error = static_cast<int>(r);
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+// Packed tokens [T][H][d] bf16 as a {d, H, T} map: a box of 64 columns x 1
+// head x 128 tokens lands in shared memory as the same 128-row tile.
+int encode_varlen_map(CUtensorMap* map, const void* ptr, int T, int H, int d) {
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -416,6 +440,70 @@ int fa_testing_fwd_starved(const void* q, const void* k, const void* v, void* o,
   if (timeout_ns == 0 || timeout_ns > kWaitTimeoutNs) return FA_ERR_INVALID_ARGUMENT;
   return launch_fwd(q, k, v, o, lse, B, H, N, N, d, scale, causal, block_mask, cuda_stream,
                     timeout_ns, 1);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int total_q,
+                  int total_k, int max_seqlen_q, int d, float scale, int causal,
+                  void* cuda_stream) {
+  if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARGUMENT;
+  if (B < 1 || H < 1 || total_q < 1 || total_k < 1 || max_seqlen_q < 1) return FA_ERR_INVALID_ARGUMENT;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARGUMENT;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
+    return FA_ERR_INVALID_ARGUMENT;
+  if (o == q || o == k || o == v) return FA_ERR_INVALID_ARGUMENT;
+  const long long bh = (long long)B * H;
+  const long long nqt = (max_seqlen_q + fa::kBM - 1) / fa::kBM;
+  const long long npairs = (nqt + 1) / 2;
+  if (bh * npairs > INT32_MAX || (long long)total_q * H > INT32_MAX) return FA_ERR_UNSUPPORTED;
+
+  DeviceState* st = nullptr;
+  int rc = get_device_state(&st);
+  if (rc != FA_OK) return rc;
+  for (const void* ptr : std::initializer_list<const void*>{q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k})
+    if (!is_device_pointer(ptr)) return FA_ERR_INVALID_ARGUMENT;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+
+  fa::KernelParams p;
+  std::memset(&p, 0, sizeof(p));
+  if ((rc = encode_varlen_map(&p.tm_q, q, total_q, H, d)) != FA_OK) return rc;
+  if ((rc = encode_varlen_map(&p.tm_k, k, total_k, H, d)) != FA_OK) return rc;
+  if ((rc = encode_varlen_map(&p.tm_v, v, total_k, H, d)) != FA_OK) return rc;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.mask = nullptr;
+  p.Nq = max_seqlen_q;
+  p.Nk = total_k;
+  p.nqt = (int)nqt;
+  p.nkt = (total_k + fa::kBN - 1) / fa::kBN;
+  p.causal_off = 0;
+  p.npairs = (int)npairs;
+  p.bh = (int)bh;
+  p.items = (int)(bh * npairs);
+  p.splits = 1;
+  p.kt_per_split = p.nkt;
+  p.causal = causal;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.timeout_ns = kWaitTimeoutNs;
+  p.status = st->status_word;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.heads = H;
+  p.total_q = total_q;
+  p.total_k = total_k;
+
+  const int grid = p.items < st->num_sms ? p.items : st->num_sms;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  if (d == 64)
+    fa::fa_fwd_kernel<64, true><<<grid, fa::kThreads, fa::Cfg<64>::kSmemBytes, stream>>>(p);
+  else
+    fa::fa_fwd_kernel<128, true><<<grid, fa::kThreads, fa::Cfg<128>::kSmemBytes, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return FA_OK;
 }
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,

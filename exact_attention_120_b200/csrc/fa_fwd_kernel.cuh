@@ -91,7 +91,81 @@ struct KernelParams {
   int kt_per_split;
   float* part_o;    // [splits][B*H*Nq][D]
   float* part_lse;  // [splits][B*H*Nq]
+  // Variable-length batches (the kernel's kVarlen instantiation): q, k, v and o
+  // are packed tokens [T][H][D]; sequence b owns token rows
+  // [cu_q[b], cu_q[b+1]) of the queries and [cu_k[b], cu_k[b+1]) of the keys;
+  // lse is [H][total_q].  Nq / Nk / nqt / nkt then hold the maxima over the
+  // batch and only bound the work grid.
+  const int* cu_q;
+  const int* cu_k;
+  int heads;
+  int total_q;
+  int total_k;
 };
+
+// Sizes of the (b, h) problem a work unit belongs to.  Dense batches: every
+// head has the kernel-wide sizes, read straight from the kernel parameters.
+// Variable-length batches: read from the sequence offsets, clamped to
+// [0, total] and made non-decreasing, so that any offsets keep every access
+// inside the buffers.
+struct SeqDense {
+  const KernelParams& p;
+  __device__ int nq() const { return p.Nq; }
+  __device__ int nk() const { return p.Nk; }
+  __device__ int nqt() const { return p.nqt; }
+  __device__ int nkt() const { return p.nkt; }
+  __device__ int causal_off() const { return p.causal_off; }  // nk - nq
+  __device__ int q0() const { return 0; }  // first token row (variable-length layout)
+  __device__ int k0() const { return 0; }
+  __device__ int h() const { return 0; }
+};
+
+struct SeqVar {
+  int nq_, nk_, nqt_, nkt_, q0_, k0_, h_;
+  __device__ int nq() const { return nq_; }
+  __device__ int nk() const { return nk_; }
+  __device__ int nqt() const { return nqt_; }
+  __device__ int nkt() const { return nkt_; }
+  __device__ int causal_off() const { return nk_ - nq_; }
+  __device__ int q0() const { return q0_; }
+  __device__ int k0() const { return k0_; }
+  __device__ int h() const { return h_; }
+};
+
+template <bool kVarlen>
+__device__ __forceinline__ auto seq_of(const KernelParams& p, int bh) {
+  if constexpr (!kVarlen) {
+    return SeqDense{p};
+  } else {
+    const int b = bh / p.heads;
+    const int qa = min(max(__ldg(p.cu_q + b), 0), p.total_q);
+    const int qb = min(max(__ldg(p.cu_q + b + 1), qa), p.total_q);
+    const int ka = min(max(__ldg(p.cu_k + b), 0), p.total_k);
+    const int kb = min(max(__ldg(p.cu_k + b + 1), ka), p.total_k);
+    SeqVar s;
+    s.h_ = bh - b * p.heads;
+    s.q0_ = qa;
+    s.k0_ = ka;
+    s.nq_ = qb - qa;
+    s.nk_ = kb - ka;
+    s.nqt_ = (s.nq_ + kBM - 1) / kBM;
+    s.nkt_ = (s.nk_ + kBN - 1) / kBN;
+    return s;
+  }
+}
+
+// TMA coordinates (y, z) of a 128-row tile starting at sequence row `row`:
+// dense maps are {D, N, B*H}, variable-length maps {D, H, T}.
+template <bool kVarlen>
+__device__ __forceinline__ void tile_coords(int row, int bh, int h, int tok0, int& y, int& z) {
+  if constexpr (kVarlen) {
+    y = h;
+    z = tok0 + row;
+  } else {
+    y = row;
+    z = bh;
+  }
+}
 
 template <int D>
 struct Cfg {
@@ -182,25 +256,29 @@ __device__ __forceinline__ void decode_item(const KernelParams& p, int w, int& b
 }
 
 // Largest key index query tile qt can see under the causal rule (may be < 0).
-__device__ __forceinline__ int causal_last_key(const KernelParams& p, int qt) {
-  return min(qt * kBM + kBM - 1, p.Nq - 1) + p.causal_off;
+template <class Seq>
+__device__ __forceinline__ int causal_last_key(const Seq& sq, int qt) {
+  return min(qt * kBM + kBM - 1, sq.nq() - 1) + sq.causal_off();
 }
 
 // Number of key tiles to scan for query tile qt: all of them, or under the
 // causal rule those up to the tile of its last visible key.
-__device__ __forceinline__ int key_tile_end(const KernelParams& p, int qt) {
-  if (!p.causal) return p.nkt;
-  const int last = causal_last_key(p, qt);
-  return last < 0 ? 0 : min(p.nkt, last / kBN + 1);
+template <class Seq>
+__device__ __forceinline__ int key_tile_end(const KernelParams& p, const Seq& sq, int qt) {
+  if (!p.causal) return sq.nkt();
+  const int last = causal_last_key(sq, qt);
+  return last < 0 ? 0 : min(sq.nkt(), last / kBN + 1);
 }
 
 // Bit l set <=> key tile j0 + l, which must lie in [jlo, jhi), is visible to
-// query tile qt (whole warp calls).
-__device__ __forceinline__ uint32_t keep_bits(const KernelParams& p, int bh, int qt, int j0,
-                                              int lane, int jlo, int jhi) {
+// query tile qt (whole warp calls).  The block mask (dense batches only) is
+// indexed with the kernel-wide tile counts.
+template <class Seq>
+__device__ __forceinline__ uint32_t keep_bits(const KernelParams& p, const Seq& sq, int bh, int qt,
+                                              int j0, int lane, int jlo, int jhi) {
   const int j = j0 + lane;
-  bool k = (qt < p.nqt) && (j >= jlo) && (j < jhi);
-  if (k && p.causal) k = j * kBN <= causal_last_key(p, qt);
+  bool k = (qt < sq.nqt()) && (j >= jlo) && (j < jhi);
+  if (k && p.causal) k = j * kBN <= causal_last_key(sq, qt);
   if (k && p.mask != nullptr) k = p.mask[((size_t)bh * p.nqt + qt) * p.nkt + j] != 0;
   return __ballot_sync(0xffffffffu, k);
 }
@@ -356,7 +434,7 @@ __device__ __forceinline__ bool mma_slot_step(const MmaCtx<D>& c, const KernelPa
   return true;
 }
 
-template <int D>
+template <int D, bool kVarlen = false>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ KernelParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -425,21 +503,25 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     for (int w = blockIdx.x; w < p.items && ok && !p.starve_producer; w += gridDim.x) {
       int bh, pair, split;
       decode_item(p, w, bh, pair, split);
+      const auto sq = seq_of<kVarlen>(p, bh);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
-      const int nvalid = (qt1 < p.nqt) ? 2 : 1;
-      const int jb = split * p.kt_per_split, je = min(p.nkt, jb + p.kt_per_split);
+      if (kVarlen && qt0 >= sq.nqt()) continue;  // past this sequence's end
+      const int nvalid = (qt1 < sq.nqt()) ? 2 : 1;
+      const int jb = split * p.kt_per_split, je = min(sq.nkt(), jb + p.kt_per_split);
       ok = wait_warp(bQEmpty, (nq & 1u) ^ 1u, abort_flag, p);
       if (ok && ptx::elect_one()) {
         ptx::mbar_arrive_expect_tx(bQFull, nvalid * C::kTileBytes);
-        for (int q = 0; q < nvalid; ++q)
+        for (int q = 0; q < nvalid; ++q) {
+          int y, z;
+          tile_coords<kVarlen>((qt0 + q) * kBM, bh, sq.h(), sq.q0(), y, z);
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            ptx::tma_load_3d(sQ + q * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q, bQFull, bx * 64,
-                             (qt0 + q) * kBM, bh);
+            ptx::tma_load_3d(sQ + q * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q, bQFull, bx * 64, y, z);
+        }
       }
       ++nq;
-      const int jend = min(je, key_tile_end(p, qt0 + nvalid - 1));
+      const int jend = min(je, key_tile_end(p, sq, qt0 + nvalid - 1));
       for (int j0 = jb & ~31; j0 < jend && ok; j0 += 32) {
-        uint32_t u = keep_bits(p, bh, qt0, j0, lane, jb, je) | keep_bits(p, bh, qt1, j0, lane, jb, je);
+        uint32_t u = keep_bits(p, sq, bh, qt0, j0, lane, jb, je) | keep_bits(p, sq, bh, qt1, j0, lane, jb, je);
         while (u != 0 && ok) {
           const int j = j0 + __ffs(u) - 1;
           u &= u - 1;
@@ -451,9 +533,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
               if (ptx::elect_one()) {
                 ptx::mbar_arrive_expect_tx(bFull(slot), C::kTileBytes);
                 const CUtensorMap* map = t == 0 ? &p.tm_k : &p.tm_v;
+                int y, z;
+                tile_coords<kVarlen>(j * kBN, bh, sq.h(), sq.k0(), y, z);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
                   ptx::tma_load_3d(sRing + slot * C::kTileBytes + bx * C::kBoxBytes, map,
-                                   bFull(slot), bx * 64, j * kBN, bh);
+                                   bFull(slot), bx * 64, y, z);
               }
               ++it;
             }
@@ -478,19 +562,21 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
       int bh, pair, split;
       decode_item(p, w, bh, pair, split);
+      const auto sq = seq_of<kVarlen>(p, bh);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
-      const bool valid1 = qt1 < p.nqt;
-      const int jb = split * p.kt_per_split, je = min(p.nkt, jb + p.kt_per_split);
+      if (kVarlen && qt0 >= sq.nqt()) continue;
+      const bool valid1 = qt1 < sq.nqt();
+      const int jb = split * p.kt_per_split, je = min(sq.nkt(), jb + p.kt_per_split);
       slot0.begin_unit(true);
       slot1.begin_unit(valid1);
       int64_t prev_v = -1;
       ok = wait_warp(bQFull, nq & 1u, abort_flag, p);
       ptx::tc_fence_after();
       ++nq;
-      const int jend = min(je, key_tile_end(p, valid1 ? qt1 : qt0));
+      const int jend = min(je, key_tile_end(p, sq, valid1 ? qt1 : qt0));
       for (int j0 = jb & ~31; j0 < jend && ok; j0 += 32) {
-        const uint32_t k0 = keep_bits(p, bh, qt0, j0, lane, jb, je);
-        const uint32_t k1 = keep_bits(p, bh, qt1, j0, lane, jb, je);
+        const uint32_t k0 = keep_bits(p, sq, bh, qt0, j0, lane, jb, je);
+        const uint32_t k1 = keep_bits(p, sq, bh, qt1, j0, lane, jb, je);
         uint32_t u = k0 | k1;
         while (u != 0 && ok) {
           const int l = __ffs(u) - 1;
@@ -561,16 +647,17 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
       int bh, pair, split;
       decode_item(p, w, bh, pair, split);
+      const auto sq = seq_of<kVarlen>(p, bh);
       const int qt = 2 * pair + q;
-      const int jb = split * p.kt_per_split, je = min(p.nkt, jb + p.kt_per_split);
-      if (qt >= p.nqt) continue;
+      const int jb = split * p.kt_per_split, je = min(sq.nkt(), jb + p.kt_per_split);
+      if (qt >= sq.nqt()) continue;
       const int row = qt * kBM + row_in_tile;  // query row within the head
       float m_ref = -INFINITY;  // reference max, in units of c * score
       float l = 0.f;            // sum of bf16-rounded 2^(c s - m_ref)
       int n = 0;                // tiles processed
-      const int jend = min(je, key_tile_end(p, qt));
+      const int jend = min(je, key_tile_end(p, sq, qt));
       for (int j0 = jb & ~31; j0 < jend && ok; j0 += 32) {
-        uint32_t kb = keep_bits(p, bh, qt, j0, lane, jb, je);
+        uint32_t kb = keep_bits(p, sq, bh, qt, j0, lane, jb, je);
         while (kb != 0 && ok) {
           const int j = j0 + __ffs(kb) - 1;
           kb &= kb - 1;
@@ -592,8 +679,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           // Mask: keys past the causal diagonal and past the end of the
           // sequence (lim = last visible column of this tile, may be < 0).
           int lim = 127;
-          if (p.causal) lim = min(lim, row + p.causal_off - j * kBN);
-          lim = min(lim, p.Nk - j * kBN - 1);
+          if (p.causal) lim = min(lim, row + sq.causal_off() - j * kBN);
+          lim = min(lim, sq.nk() - j * kBN - 1);
           if (lim < 127) {
 #pragma unroll
             for (int c = 0; c < 128; ++c)
@@ -691,7 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       // scores only add 2^-125 through the FMA-pipe exp2): O = 0, lse = -inf.
       const bool seen = m_ref != -INFINITY && l > 0.f;
       const float inv = seen ? 1.f / l : 0.f;
-      const bool in_range = row < p.Nq;
+      // Sizes again (not held in registers across the tile loop).
+      const auto se = seq_of<kVarlen>(p, bh);
+      const bool in_range = row < se.nq();
       if (p.splits > 1) {
         // Partial result of this key slice: normalised O (fp32) and its lse.
         const size_t prow = (size_t)split * p.bh * p.Nq + (size_t)bh * p.Nq + (in_range ? row : 0);
@@ -716,7 +805,12 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         if (in_range)
           p.part_lse[prow] = seen ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
       } else {
-      uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D);
+      // O row and lse element of this query: [B*H][Nq] rows, or token-major
+      // [T][H] rows with lse [H][T] for variable-length batches.
+      const int r = in_range ? row : 0;
+      const size_t orow_i = kVarlen ? (size_t)(se.q0() + r) * p.heads + se.h() : (size_t)bh * p.Nq + r;
+      const size_t lse_i = kVarlen ? (size_t)se.h() * p.total_q + se.q0() + r : (size_t)bh * p.Nq + r;
+      uint4* orow = reinterpret_cast<uint4*>(p.o + orow_i * D);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t t[32];
@@ -738,8 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         }
       }
       if (in_range)
-        p.lse[(size_t)bh * p.Nq + row] =
-            seen ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        p.lse[lse_i] = seen ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(bOEmpty(q));

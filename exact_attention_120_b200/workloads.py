@@ -18,6 +18,7 @@ std 3 gives score std ~9 at scale 1/sqrt(d), variance 3 only ~3).
 
 from __future__ import annotations
 
+import itertools
 import math
 from dataclasses import dataclass, field
 
@@ -114,3 +115,74 @@ def algorithmic_bytes(B, H, N, d):
     """HBM bytes of one forward pass if every tensor moves once:
     bf16 Q, K, V read and O written (8*N*d per head) plus fp32 lse (4*N)."""
     return float(B * H * (8 * N * d + 4 * N))
+
+
+# ---------------------------------------------------------------- varlen ---
+# Variable-length batches: sequences packed token-major ([T, H, d]) with int32
+# offsets cu = [0, n_0, n_0 + n_1, ...].  The length mix is log-uniform, the
+# shape of a batch of documents or prompts of very different sizes.
+
+
+@dataclass(frozen=True)
+class VarlenWorkload:
+    name: str
+    B: int          # sequences
+    H: int
+    d: int
+    min_len: int
+    max_len: int
+    causal: bool = True
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def describe(self) -> str:
+        return (f"B={self.B} sequences, lengths log-uniform in [{self.min_len},{self.max_len}], "
+                f"H={self.H}, d={self.d}, {'causal' if self.causal else 'full'}")
+
+
+VARLEN_WORKLOADS = {
+    "varlen_mix": VarlenWorkload("varlen_mix", 32, 16, 128, 128, 8192, causal=True, seed=5),
+}
+
+
+def varlen_lengths(B, lo, hi, seed):
+    """B integer lengths, log-uniform in [lo, hi]."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    u = torch.rand(B, generator=g, dtype=torch.float64)
+    n = torch.exp(math.log(lo) + u * (math.log(hi) - math.log(lo)))
+    return [int(x) for x in n.round().clamp(lo, hi).tolist()]
+
+
+def make_varlen(lengths_q, lengths_k, H, d, seed, qk_std=1.0):
+    """Packed bf16 q [Tq, H, d], k, v [Tk, H, d] and int32 offsets cu_q, cu_k
+    (CPU), drawn like make_qkv in the order q, k, v."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    Tq, Tk = int(sum(lengths_q)), int(sum(lengths_k))
+    q = (torch.randn((Tq, H, d), generator=g) * qk_std).to(torch.bfloat16)
+    k = (torch.randn((Tk, H, d), generator=g) * qk_std).to(torch.bfloat16)
+    v = torch.randn((Tk, H, d), generator=g).to(torch.bfloat16)
+    cu = lambda ls: torch.tensor([0] + list(itertools.accumulate(ls)), dtype=torch.int32)  # noqa: E731
+    return q, k, v, cu(lengths_q), cu(lengths_k)
+
+
+def make_varlen_inputs(w: VarlenWorkload):
+    lens = varlen_lengths(w.B, w.min_len, w.max_len, w.seed)
+    return (lens,) + make_varlen(lens, lens, w.H, w.d, w.seed + 1)
+
+
+def varlen_flops(lengths_q, lengths_k, H, d, causal):
+    """Useful FLOPs: 4 d per visible (query, key) pair, per head (causal: key
+    j visible to query i iff j <= i + nk - nq)."""
+    f = 0.0
+    for nq, nk in zip(lengths_q, lengths_k):
+        if causal:
+            off = nk - nq
+            # sum over i of clamp(i + off + 1, 0, nk)
+            vis = sum(min(max(i + off + 1, 0), nk) for i in range(nq))
+        else:
+            vis = nq * nk
+        f += 4.0 * d * H * vis
+    return f

@@ -168,6 +168,36 @@ FA_API int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, v
 FA_API int fa_fwd_splitkv_heuristic(int B, int H, int Nq, int Nk);
 
 /*
+ * Variable-length batch: B independent attention problems of different
+ * lengths in one launch, the layout of packed token streams.  Sequence b
+ * owns query token rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key/value
+ * rows [cu_seqlens_k[b], cu_seqlens_k[b+1]); its queries attend to its own
+ * keys only, each sequence computed exactly as fa_fwd_qk computes one head
+ * (same softmax, same bottom-right causal rule j <= i + (nk_b - nq_b), an
+ * empty sequence or a query row with no visible key gives O = 0,
+ * lse = -inf).  The pages treat one sequence; batching unequal lengths
+ * without padding is this library's extension of the same loop.
+ *
+ * q, o: bf16 [total_q, H, d]; k, v: bf16 [total_k, H, d] (token-major, d
+ * fastest); lse: fp32 [H, total_q].  cu_seqlens_q / cu_seqlens_k: int32
+ * device arrays of B+1 non-decreasing offsets starting at 0 and ending at
+ * total_q / total_k.  max_seqlen_q must be >= every query length: rows past
+ * it are not computed.  Offsets outside [0, total] are clamped on the device
+ * (so no access leaves the buffers), but such a batch has no defined result.
+ * No block mask.  All pointers device memory owned by the caller, 16-byte
+ * aligned (lse, cu_seqlens: 4).  Asynchronous on cuda_stream.
+ *
+ * Returns FA_OK, FA_ERR_INVALID_ARGUMENT (null, host or misaligned pointer,
+ * B, H, total_q, total_k or max_seqlen_q < 1, bad scale or causal, o
+ * aliasing an input), FA_ERR_UNSUPPORTED (d not 64 or 128, no sm_100
+ * device, more than 2^31 work units or query rows x H) or FA_ERR_CUDA.
+ */
+FA_API int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H,
+                         int total_q, int total_k, int max_seqlen_q, int d, float scale,
+                         int causal, void* cuda_stream);
+
+/*
  * Backward pass: dQ, dK, dV of the forward above for the upstream gradient
  * dO.  The scores are recomputed from q, k and the forward's lse, not stored
  * ("理解 Flash Attention", section "瓦片注意力计算"), with P = exp(S - lse),

@@ -76,3 +76,10 @@ def test_splitkv_workspace_size(lib):
     assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 10, 300, 64, 100) == 3 * 10 * 65 * 4
     assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 10, 300, 64, 1) == 0
     assert fa.fa_fwd_splitkv_workspace_bytes(1, 1, 10, 300, 64, 0) == 0
+
+
+def test_every_public_name_exists():
+    import exact_attention_120_b200 as fa
+
+    missing = [n for n in fa.__all__ if not hasattr(fa, n)]
+    assert not missing, missing
