@@ -26,6 +26,9 @@ Modules:
 * ``backward``       -- dQ, dK, dV by the chain rule through the definition.
 * ``varlen``         -- variable-length batches: independent sequences packed
                         token-major without padding.
+* ``fp8``            -- the E4M3 format written out, attention of the real
+                        values 8-bit codes stand for, and the weighted spread
+                        of V that bounds the effect of rounding P.
 
 Every function here is pinned by ``tests/test_oracle.py`` to closed forms,
 invariants and the pages' worked example; see that file's header.
@@ -41,3 +44,4 @@ from .attention import (  # noqa: F401
 from .brute import attention_brute  # noqa: F401
 from .backward import attention_bwd_ref, softmax_delta  # noqa: F401
 from .varlen import attention_varlen_ref  # noqa: F401
+from .fp8 import attention_fp8_ref, e4m3_decode, weighted_spread  # noqa: F401
