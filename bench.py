@@ -22,7 +22,8 @@ alone as the reference arm.
 ``--pass bwd`` times fa_bwd (dQ, dK, dV from the forward's O and lse) on the
 same workload instead, credited with 2.5x the forward's FLOPs.  ``--pass
 varlen`` times fa_fwd_varlen on varlen_mix (32 causal sequences of 128 to 8192
-tokens packed without padding, H=16, d=128).
+tokens packed without padding, H=16, d=128).  ``--pass fp8`` times fa_fwd_fp8
+on the workload's shape with Q, K, V quantised to E4M3.
 
 Multi-GPU (launched by torchrun): ranks share nothing on the data path; each
 rank runs the full workload shape on its own batch slice (weak scaling).
@@ -46,8 +47,8 @@ sys.path.insert(0, ROOT)
 
 from exact_attention_120_b200 import sharding  # noqa: E402
 from exact_attention_120_b200.workloads import (VARLEN_WORKLOADS, WORKLOADS, algorithmic_bytes,  # noqa: E402
-                                                make_inputs, make_varlen_inputs, useful_flops,
-                                                varlen_flops)
+                                                make_inputs, make_qkv_fp8, make_varlen_inputs,
+                                                useful_flops, varlen_flops)
 
 METRIC = "fused attention fwd TFLOP/s (bf16, causal & full) and % of dense BF16 peak"
 UNIT = "TFLOP/s"
@@ -470,6 +471,71 @@ class VarlenJob(FwdJob):
                           f"{t_total:.1f} s"}
 
 
+class Fp8Job(FwdJob):
+    """One step = one fa_fwd_fp8 launch: the workload's shape with Q, K, V
+    quantised to E4M3 (one scale per tensor), O in bf16."""
+
+    name = "fp8"
+    metric = "fused attention fwd TFLOP/s, 8-bit E4M3 inputs, and % of dense FP8 peak"
+    peak_ratio = 2.0  # dense fp8 / dense bf16, nominal (4.5 / 2.25 PFLOP/s)
+
+    def __init__(self, fa, torch, w, dev, stream):
+        if w.d != 128 or w.sparse_p is not None:
+            raise SystemExit("--pass fp8 runs d=128 workloads without a block mask")
+        self.fa, self.w, self.stream = fa, w, stream
+        (q8, k8, v8), self.descales = make_qkv_fp8(w.B, w.H, w.N, w.d, w.seed, w.qk_std, w.v_std)
+        self.flops = useful_flops(w.B, w.H, w.N, w.d, w.causal, None)
+        self.q, self.k, self.v = q8, k8, v8
+        self.qd, self.kd, self.vd = q8.to(dev), k8.to(dev), v8.to(dev)
+        self.od = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=dev)
+        self.ld = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        self.mask = None
+        self.launches_per_step = 1
+
+    def launch(self):
+        w, fa = self.w, self.fa
+        st = fa.fa_fwd_fp8(self.qd.data_ptr(), self.kd.data_ptr(), self.vd.data_ptr(),
+                           self.od.data_ptr(), self.ld.data_ptr(), w.B, w.H, w.N, w.N, w.d, w.scale,
+                           int(w.causal), None, *self.descales, self.stream.cuda_stream)
+        if st != fa.FA_OK:
+            raise fa.FaError(st, "fa_fwd_fp8")
+
+    def host_buffers(self):
+        torch = __import__("torch")
+        self.hin = [t.pin_memory() for t in (self.q, self.k, self.v)]
+        self.hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (self.od, self.ld)]
+        return (sum(t.numel() * t.element_size() for t in self.hin),
+                sum(t.numel() * t.element_size() for t in self.hout))
+
+    def e2e_step(self):
+        for d, h in zip((self.qd, self.kd, self.vd), self.hin):
+            d.copy_(h, non_blocking=True)
+        w = self.w
+        self.fa.attention_forward_fp8(self.qd, self.kd, self.vd, *self.descales, causal=w.causal,
+                                      scale=w.scale, out=self.od, lse=self.ld)
+        for h, d in zip(self.hout, (self.od, self.ld)):
+            h.copy_(d, non_blocking=True)
+
+    def algorithmic_bytes(self):
+        # 1-byte Q, K, V read, bf16 O and fp32 lse written.
+        w = self.w
+        return float(w.B * w.H * (5 * w.N * w.d + 4 * w.N))
+
+    def cpu_baseline(self, args):
+        import oracle
+
+        torch = __import__("torch")
+        w = self.w
+        qd, kd, vd = self.descales
+        f64 = lambda t, s: torch.from_numpy(oracle.e4m3_decode(t.numpy()) * s)  # noqa: E731
+        qf, kf, vf = f64(self.q, qd), f64(self.k, kd), f64(self.v, vd)
+        f, t, rows = oracle_sample(w, qf.numpy(), kf.numpy(), vf.numpy(), None, args.cpu_rows,
+                                   budget_s=args.cpu_budget)
+        return {"value": f / t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{rows} query rows of {w.name} (E4M3 inputs decoded exactly), {t:.1f} s "
+                          f"of float64 NumPy/BLAS oracle"}
+
+
 def varlen_config(w, job, world):
     return {"workload": f"{w.name}: {w.describe()}, scale 1/sqrt(d), seed {w.seed}",
             "B": w.B, "H": w.H, "d": w.d, "causal": w.causal, "total_tokens": int(job.qd.shape[0]),
@@ -492,7 +558,11 @@ def run_ours(args, info):
     fa.load_library()
 
     stream = torch.cuda.current_stream(dev)
-    if args.pass_ == "varlen":
+    if args.pass_ == "fp8":
+        w = WORKLOADS[args.workload]
+        job = Fp8Job(fa, torch, dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank)),
+                     dev, stream)
+    elif args.pass_ == "varlen":
         w = VARLEN_WORKLOADS["varlen_mix"]
         job = VarlenJob(fa, torch, dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank)),
                         dev, stream)
@@ -557,6 +627,8 @@ def run_ours(args, info):
         return 0
 
     peak, peak_sus, peak_src = load_peaks()
+    ratio = getattr(job, "peak_ratio", 1.0)
+    peak, peak_sus = peak * ratio, peak_sus * ratio
     achieved = flops / (ms_step * 1e-3) / 1e12  # one call per step
     value = info.world_size * achieved
     cpu = None
@@ -566,14 +638,16 @@ def run_ours(args, info):
     line = {
         "metric": job.metric, "value": value, "unit": UNIT, "n_gpus": info.world_size,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if job.name == "fp8" else "bf16",
         "data": "synthetic (seeded N(0,1) draws, bf16)",
         "config": (varlen_config(w, job, info.world_size) if job.name == "varlen"
                    else workload_config(w, info.world_size)),
         "pct_of_dense_bf16_peak": 100.0 * achieved / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": load_traffic(w.name, job.name, khash),
-                     "peak_kind": f"{peak_src} burst dense bf16",
+                     "peak_kind": (f"{peak_src} burst dense bf16" if ratio == 1.0 else
+                                   f"{peak_src} burst dense bf16 x {ratio:g} (nominal fp8/bf16 ratio)"),
                      "frac_of_sustained_peak": achieved / peak_sus,
                      "algorithmic_bytes": job.algorithmic_bytes(),
                      "flops_per_launch": flops},
@@ -597,9 +671,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="long_full", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "varlen"],
-                    help="time the forward (default), the backward pass, or the forward on the "
-                         "variable-length batch varlen_mix (--workload is then ignored)")
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd", "varlen", "fp8"],
+                    help="time the forward (default), the backward pass, the 8-bit forward, or the "
+                         "forward on the variable-length batch varlen_mix (--workload is then ignored)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-rows", type=int, default=256, help="oracle rows per timed chunk")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")

@@ -30,7 +30,8 @@ __all__ = [
     "FaError", "library_path", "load_library", "fa_fwd", "fa_fwd_stream", "fa_fwd_qk",
     "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_heuristic",
     "attention_forward_splitkv", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward",
-    "fa_device_status", "fa_fwd_varlen", "attention_forward_varlen",
+    "fa_device_status", "fa_fwd_varlen", "attention_forward_varlen", "fa_fwd_fp8",
+    "attention_forward_fp8",
     "fa_status_string", "fa_launches_per_call", "attention_forward", "FA_OK",
     "FA_ERR_INVALID_ARGUMENT", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT",
     "MASK_BLOCK",
@@ -65,6 +66,9 @@ _SIGNATURES = {
                                + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                                        ctypes.c_int, ctypes.c_void_p]),
     "fa_fwd_splitkv_heuristic": (ctypes.c_int, [ctypes.c_int] * 4),
+    "fa_fwd_fp8": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5
+                   + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p] + [ctypes.c_float] * 3
+                   + [ctypes.c_void_p]),
     "fa_fwd_varlen": (ctypes.c_int, [ctypes.c_void_p] * 7 + [ctypes.c_int] * 6
                       + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
     "fa_bwd": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
@@ -254,6 +258,12 @@ def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, to
                                         total_k, max_seqlen_q, d, scale, causal, stream)
 
 
+def fa_fwd_fp8(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, q_descale, k_descale,
+               v_descale, stream) -> int:
+    return load_library().fa_fwd_fp8(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask,
+                                     q_descale, k_descale, v_descale, stream)
+
+
 def fa_bwd_workspace_bytes(B, H, Nq) -> int:
     return load_library().fa_bwd_workspace_bytes(B, H, Nq)
 
@@ -329,4 +339,37 @@ def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
                                           float(scale), int(bool(causal)), stream)
     if st != FA_OK:
         raise FaError(st, "fa_fwd_varlen")
+    return out, lse
+
+
+def attention_forward_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal=False, block_mask=None,
+                          scale=None, out=None, lse=None, stream=None):
+    """O (bf16), lse of attention on 8-bit E4M3 inputs through the C ABI (fa_fwd_fp8).
+
+    q8: CUDA uint8 or float8_e4m3fn [B, H, Nq, 128]; k8, v8: [B, H, Nk, 128];
+    the codes stand for q_descale * q8 etc.  scale defaults to 1/sqrt(d).
+    """
+    import torch
+
+    B, H, Nq, d = q8.shape
+    Nk = k8.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    for t in (q8, k8, v8):
+        if t.element_size() != 1 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q8, k8, v8 must be contiguous CUDA 8-bit tensors")
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q8.device)
+    mask_ptr = None if block_mask is None else block_mask.data_ptr()
+    if stream is None:
+        stream = torch.cuda.current_stream(q8.device).cuda_stream
+    with torch.cuda.device(q8.device):
+        st = load_library().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                                       lse.data_ptr(), B, H, Nq, Nk, d, float(scale), int(bool(causal)),
+                                       mask_ptr, float(q_descale), float(k_descale), float(v_descale),
+                                       stream)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_fp8")
     return out, lse

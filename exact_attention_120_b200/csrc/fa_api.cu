@@ -58,16 +58,19 @@ int setup_device(int dev, DeviceState& st) {
   if (e != cudaSuccess) return cuda_fail(e);
   if (prop.major != 10 || prop.minor != 0) return FA_ERR_UNSUPPORTED;  // sm_100 only
   st.num_sms = prop.multiProcessorCount;
-  e = cudaFuncSetAttribute(fa::fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(fa::fa_fwd_kernel<fa::Cfg<64>>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            fa::Cfg<64>::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaFuncSetAttribute(fa::fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(fa::fa_fwd_kernel<fa::Cfg<128>>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            fa::Cfg<128>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa::fa_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(fa::fa_fwd_kernel<fa::Cfg<128, true>>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fa::Cfg<128, true>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fa::fa_fwd_kernel<fa::Cfg<64>, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::Cfg<64>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa::fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(fa::fa_fwd_kernel<fa::Cfg<128>, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::Cfg<128>::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -125,13 +128,16 @@ bool is_device_pointer(const void* p) {
   return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
 }
 
-// [B*H][N][d] bf16, boxes of 64 columns x 128 rows, 128-byte swizzle.
-int encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
+// [B*H][N][d] bf16 (elt_bytes 2) or 8-bit (elt_bytes 1), boxes of 128 bytes
+// x 128 rows, 128-byte swizzle.
+int encode_qkv_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int elt_bytes = 2) {
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * elt_bytes, (cuuint64_t)N * d * elt_bytes};
+  const cuuint32_t box[3] = {(cuuint32_t)(128 / elt_bytes), 128, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+  const CUtensorMapDataType dt =
+      elt_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = g_encode(map, dt, 3, const_cast<void*>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -187,9 +193,15 @@ size_t splitkv_workspace_bytes(size_t rows, int d, int splits) {
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
                void* cuda_stream, unsigned long long timeout_ns, int starve_producer,
-               int num_splits = 1, void* workspace = nullptr, size_t workspace_bytes = 0) {
+               int num_splits = 1, void* workspace = nullptr, size_t workspace_bytes = 0,
+               bool fp8 = false, float q_descale = 1.f, float k_descale = 1.f,
+               float v_descale = 1.f) {
   // ---- arguments (nothing is launched on error)
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
+  if (fp8 && !(std::isfinite(q_descale) && q_descale > 0.f && std::isfinite(k_descale) &&
+               k_descale > 0.f && std::isfinite(v_descale) && v_descale > 0.f))
+    return FA_ERR_INVALID_ARGUMENT;
+  if (fp8 && d != 128) return FA_ERR_UNSUPPORTED;
   if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARGUMENT;
   if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARGUMENT;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARGUMENT;
@@ -229,9 +241,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   // ---- parameters
   fa::KernelParams p;
   std::memset(&p, 0, sizeof(p));
-  if ((rc = encode_qkv_map(&p.tm_q, q, (int)bh, Nq, d)) != FA_OK) return rc;
-  if ((rc = encode_qkv_map(&p.tm_k, k, (int)bh, Nk, d)) != FA_OK) return rc;
-  if ((rc = encode_qkv_map(&p.tm_v, v, (int)bh, Nk, d)) != FA_OK) return rc;
+  const int eb = fp8 ? 1 : 2;
+  if ((rc = encode_qkv_map(&p.tm_q, q, (int)bh, Nq, d, eb)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_k, k, (int)bh, Nk, d, eb)) != FA_OK) return rc;
+  if ((rc = encode_qkv_map(&p.tm_v, v, (int)bh, Nk, d, eb)) != FA_OK) return rc;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.mask = block_mask;
@@ -250,7 +263,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.part_lse = p.part_o + (size_t)splits * rows * d;
   }
   p.causal = causal;
-  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.scale_log2 = (float)((double)scale * q_descale * k_descale * 1.4426950408889634074);
+  p.o_scale = v_descale;
   p.timeout_ns = timeout_ns;
   p.status = st->status_word;
   p.starve_producer = starve_producer;
@@ -258,10 +272,12 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   // ---- launch: persistent grid, one CTA per SM
   const int grid = p.items < st->num_sms ? p.items : st->num_sms;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-  if (d == 64)
-    fa::fa_fwd_kernel<64><<<grid, fa::kThreads, fa::Cfg<64>::kSmemBytes, stream>>>(p);
+  if (fp8)
+    fa::fa_fwd_kernel<fa::Cfg<128, true>><<<grid, fa::kThreads, fa::Cfg<128, true>::kSmemBytes, stream>>>(p);
+  else if (d == 64)
+    fa::fa_fwd_kernel<fa::Cfg<64>><<<grid, fa::kThreads, fa::Cfg<64>::kSmemBytes, stream>>>(p);
   else
-    fa::fa_fwd_kernel<128><<<grid, fa::kThreads, fa::Cfg<128>::kSmemBytes, stream>>>(p);
+    fa::fa_fwd_kernel<fa::Cfg<128>><<<grid, fa::kThreads, fa::Cfg<128>::kSmemBytes, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   if (splits > 1) {  // merge the slices (concatenated-softmax rule)
@@ -415,7 +431,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   p.causal = causal;
   p.scale = scale;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
-  p.timeout_ns = kWaitTimeoutNs;
+    p.timeout_ns = kWaitTimeoutNs;
   p.status = st->status_word;
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
@@ -440,6 +456,13 @@ int fa_testing_fwd_starved(const void* q, const void* k, const void* v, void* o,
   if (timeout_ns == 0 || timeout_ns > kWaitTimeoutNs) return FA_ERR_INVALID_ARGUMENT;
   return launch_fwd(q, k, v, o, lse, B, H, N, N, d, scale, causal, block_mask, cuda_stream,
                     timeout_ns, 1);
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
+               float q_descale, float k_descale, float v_descale, void* cuda_stream) {
+  return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
+                    kWaitTimeoutNs, 0, 1, nullptr, 0, true, q_descale, k_descale, v_descale);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -487,6 +510,7 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   p.kt_per_split = p.nkt;
   p.causal = causal;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.o_scale = 1.0f;
   p.timeout_ns = kWaitTimeoutNs;
   p.status = st->status_word;
   p.cu_q = cu_seqlens_q;
@@ -498,9 +522,9 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   const int grid = p.items < st->num_sms ? p.items : st->num_sms;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   if (d == 64)
-    fa::fa_fwd_kernel<64, true><<<grid, fa::kThreads, fa::Cfg<64>::kSmemBytes, stream>>>(p);
+    fa::fa_fwd_kernel<fa::Cfg<64>, true><<<grid, fa::kThreads, fa::Cfg<64>::kSmemBytes, stream>>>(p);
   else
-    fa::fa_fwd_kernel<128, true><<<grid, fa::kThreads, fa::Cfg<128>::kSmemBytes, stream>>>(p);
+    fa::fa_fwd_kernel<fa::Cfg<128>, true><<<grid, fa::kThreads, fa::Cfg<128>::kSmemBytes, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return FA_OK;

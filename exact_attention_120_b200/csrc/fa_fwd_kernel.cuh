@@ -76,7 +76,8 @@ struct KernelParams {
   int bh;      // B * H
   int items;   // bh * npairs
   int causal;
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (8-bit inputs: times the Q and K dequantisation scales)
+  float o_scale;     // multiplies O: 1, or the V dequantisation scale for 8-bit inputs
   unsigned long long timeout_ns;
   int* status;  // device status word
   // Test hook of the failure-detection test: when set, the TMA producer issues
@@ -167,13 +168,19 @@ __device__ __forceinline__ void tile_coords(int row, int bh, int h, int tok0, in
   }
 }
 
-template <int D>
+template <int D_, bool kFp8_ = false>
 struct Cfg {
-  static_assert(D == 64 || D == 128, "head dim 64 or 128");
-  static constexpr int kBoxes = D / 64;          // 64-column TMA boxes per tile
-  static constexpr int kBoxBytes = 128 * 128;    // 128 rows x 128 B
-  static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kStages = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int kD = D_;
+  static constexpr bool kFp8 = kFp8_;  // e4m3 Q, K, V (kind::f8f6f4); bf16 otherwise
+  static_assert(D_ == 64 || D_ == 128, "head dim 64 or 128");
+  static_assert(!kFp8_ || D_ == 128, "8-bit inputs: head dim 128 (one 128-byte swizzle row)");
+  static constexpr int kEltBytes = kFp8_ ? 1 : 2;
+  static constexpr int kBoxCols = 128 / kEltBytes;          // elements per 128-byte box row
+  static constexpr int kBoxes = D_ * kEltBytes / 128;       // TMA boxes per tile
+  static constexpr int kBoxBytes = 128 * 128;               // 128 rows x 128 B
+  static constexpr int kTileBytes = 128 * D_ * kEltBytes;
+  static constexpr int kKStep = kFp8_ ? 32 : 16;            // K of one MMA instruction
+  static constexpr int kStages = (kTileBytes == 32768) ? 4 : 8;  // K/V ring slots
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
@@ -183,13 +190,22 @@ struct Cfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   // Tensor memory columns.  At d = 128, S_0, S_1, O_0, O_1 fill all 512 and P_q
-  // is written over S_q.  At d = 64 there is room for P_q of its own, so the
-  // next S_q can be computed while the softmax of the current one still runs.
-  static constexpr bool kSeparateP = (D == 64);
+  // is written over S_q (bf16: 64 columns, e4m3: 32).  At d = 64 there is room
+  // for P_q of its own, so the next S_q can be computed while the softmax of
+  // the current one still runs.
+  static constexpr bool kSeparateP = (D_ == 64);
   static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO0 = 256;
   static constexpr uint32_t kTmemO1 = kSeparateP ? 320 : 384;
   static constexpr uint32_t kTmemP0 = kSeparateP ? 384 : kTmemS0;
   static constexpr uint32_t kTmemP1 = kSeparateP ? 448 : kTmemS1;
+  // Online-softmax reference: the reference max moves when the running max
+  // exceeds it by more than kRescale (log2 units), and P = 2^(x - m_ref +
+  // kPShift).  bf16 P: shift 0, P <= 2^8.  e4m3 P: the exponent range is
+  // narrow (normal from 2^-6, largest 448), so the reference moves sooner and
+  // P is shifted up by 2^4: P <= 2^8 still, while values down to 2^-18 of the
+  // reference survive the rounding.
+  static constexpr float kRescale = kFp8_ ? 4.0f : 8.0f;
+  static constexpr float kPShift = kFp8_ ? 4.0f : 0.0f;
 };
 
 // 2^x on the FMA pipe for two lanes (relieves the MUFU exp2 unit, which at
@@ -229,6 +245,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
   return (1u << 4)                           // D format: f32
          | (1u << 7)                         // A format: bf16
          | (1u << 10)                        // B format: bf16
+         | ((b_mn_major ? 1u : 0u) << 16)    // B major-ness
+         | ((uint32_t)(N >> 3) << 17)        // N / 8
+         | ((uint32_t)(M >> 4) << 24);       // M / 16
+}
+
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (format code 0), fp32
+// accumulator, A K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major) {
+  return (1u << 4)                           // D format: f32
          | ((b_mn_major ? 1u : 0u) << 16)    // B major-ness
          | ((uint32_t)(N >> 3) << 17)        // N / 8
          | ((uint32_t)(M >> 4) << 24);       // M / 16
@@ -313,19 +338,31 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
 // Barrier addresses shared by the kernel and the MMA helpers.  Layout from
 // bar0: q_full, q_empty, full[S], empty[S], s_full[2], p_full[2], o_full[2],
 // o_empty[2], p_half[2], mma_done.
-template <int D> __device__ __forceinline__ uint32_t bar_full(uint32_t bar0, int s) { return bar0 + 16 + 8u * s; }
-template <int D> __device__ __forceinline__ uint32_t bar_q(uint32_t bar0) { return bar0 + 16 + 16u * Cfg<D>::kStages; }
-template <int D> __device__ __forceinline__ uint32_t bar_s_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 8u * q; }
-template <int D> __device__ __forceinline__ uint32_t bar_p_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 16 + 8u * q; }
-template <int D> __device__ __forceinline__ uint32_t bar_o_full(uint32_t bar0, int q) { return bar_q<D>(bar0) + 32 + 8u * q; }
-template <int D> __device__ __forceinline__ uint32_t bar_o_empty(uint32_t bar0, int q) { return bar_q<D>(bar0) + 48 + 8u * q; }
+template <class C> __device__ __forceinline__ uint32_t bar_full(uint32_t bar0, int s) { return bar0 + 16 + 8u * s; }
+template <class C> __device__ __forceinline__ uint32_t bar_q(uint32_t bar0) { return bar0 + 16 + 16u * C::kStages; }
+template <class C> __device__ __forceinline__ uint32_t bar_s_full(uint32_t bar0, int q) { return bar_q<C>(bar0) + 8u * q; }
+template <class C> __device__ __forceinline__ uint32_t bar_p_full(uint32_t bar0, int q) { return bar_q<C>(bar0) + 16 + 8u * q; }
+template <class C> __device__ __forceinline__ uint32_t bar_o_full(uint32_t bar0, int q) { return bar_q<C>(bar0) + 32 + 8u * q; }
+template <class C> __device__ __forceinline__ uint32_t bar_o_empty(uint32_t bar0, int q) { return bar_q<C>(bar0) + 48 + 8u * q; }
 // P of keys [0, 64) of the tile is in tensor memory (p_full: all 128 keys).
-template <int D> __device__ __forceinline__ uint32_t bar_p_half(uint32_t bar0, int q) { return bar_q<D>(bar0) + 64 + 8u * q; }
+template <class C> __device__ __forceinline__ uint32_t bar_p_half(uint32_t bar0, int q) { return bar_q<C>(bar0) + 64 + 8u * q; }
 // Separate-P layout only: the softmax has read S_q (s_free), the PV MMAs of
 // slot q's latest P are complete (pv_done).
-template <int D> __device__ __forceinline__ uint32_t bar_s_free(uint32_t bar0, int q) { return bar_q<D>(bar0) + 80 + 8u * q; }
-template <int D> __device__ __forceinline__ uint32_t bar_pv_done(uint32_t bar0, int q) { return bar_q<D>(bar0) + 96 + 8u * q; }
-template <int D> __device__ __forceinline__ uint32_t bar_mma_done(uint32_t bar0) { return bar_q<D>(bar0) + 112; }
+template <class C> __device__ __forceinline__ uint32_t bar_s_free(uint32_t bar0, int q) { return bar_q<C>(bar0) + 80 + 8u * q; }
+template <class C> __device__ __forceinline__ uint32_t bar_pv_done(uint32_t bar0, int q) { return bar_q<C>(bar0) + 96 + 8u * q; }
+template <class C> __device__ __forceinline__ uint32_t bar_mma_done(uint32_t bar0) { return bar_q<C>(bar0) + 112; }
+
+// The MMA of the configuration's kind (kind::f16 for bf16, kind::f8f6f4 for e4m3).
+template <class C>
+__device__ __forceinline__ void mma_ss_any(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if constexpr (C::kFp8) ptx::mma_ss_f8(d, a, b, idesc, acc);
+  else ptx::mma_ss(d, a, b, idesc, acc);
+}
+template <class C>
+__device__ __forceinline__ void mma_ts_any(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if constexpr (C::kFp8) ptx::mma_ts_f8(d, a, b, idesc, acc);
+  else ptx::mma_ts(d, a, b, idesc, acc);
+}
 
 // MMA-issuer state of one query slot.
 struct MmaSlot {
@@ -345,7 +382,7 @@ struct MmaSlot {
   }
 };
 
-template <int D>
+template <class C>
 struct MmaCtx {
   uint32_t tmem, sQ, sRing;
   volatile int* abort_flag;
@@ -353,24 +390,28 @@ struct MmaCtx {
 
 // O_q += P_q V for the pending V of slot Q.  Called by the whole MMA warp
 // (warp-uniform); one elected lane issues.
-template <int D, int Q>
-__device__ __forceinline__ bool mma_issue_pv(const MmaCtx<D>& c, const KernelParams& p, MmaSlot& s,
+template <class C, int Q>
+__device__ __forceinline__ bool mma_issue_pv(const MmaCtx<C>& c, const KernelParams& p, MmaSlot& s,
                                              int64_t& v_ready, uint32_t bar0) {
-  using C = Cfg<D>;
-  constexpr uint32_t kIdescPV = idesc_bf16(128, D, true);
+  constexpr int D = C::kD;
+  constexpr uint32_t kIdescPV = C::kFp8 ? idesc_e4m3(128, D, true) : idesc_bf16(128, D, true);
+  // One MMA per kKStep keys: A = 8 tensor-memory columns of P (32 bytes per
+  // row), B = kKStep rows of V (MN-major, 128 B per row).
+  constexpr int kSteps = kBN / C::kKStep;
+  constexpr uint32_t kVStep = C::kKStep * 128;
   // Keys [0, 64) of P first: their MMAs overlap the softmax of keys [64, 128).
-  if (!wait_warp(bar_p_half<D>(bar0, Q), s.pwait & 1u, c.abort_flag, p)) return false;
+  if (!wait_warp(bar_p_half<C>(bar0, Q), s.pwait & 1u, c.abort_flag, p)) return false;
   ptx::tc_fence_after();
   const int64_t vr = s.pend;
   if (vr > v_ready) {
-    if (!wait_warp(bar_full<D>(bar0, (int)(vr % C::kStages)), (uint32_t)(vr / C::kStages) & 1u,
+    if (!wait_warp(bar_full<C>(bar0, (int)(vr % C::kStages)), (uint32_t)(vr / C::kStages) & 1u,
                    c.abort_flag, p))
       return false;
     v_ready = vr;
     ptx::tc_fence_after();
   }
   if (s.need_oe) {  // the previous unit's epilogue has read O_q
-    if (!wait_warp(bar_o_empty<D>(bar0, Q), (s.nitems - 1) & 1u, c.abort_flag, p)) return false;
+    if (!wait_warp(bar_o_empty<C>(bar0, Q), (s.nitems - 1) & 1u, c.abort_flag, p)) return false;
     s.need_oe = false;
     ptx::tc_fence_after();
   }
@@ -379,19 +420,19 @@ __device__ __forceinline__ bool mma_issue_pv(const MmaCtx<D>& c, const KernelPar
   const uint32_t tP = c.tmem + (Q ? C::kTmemP1 : C::kTmemP0);
   const uint32_t acc0 = s.npv > 0 ? 1u : 0u;
 #pragma unroll
-  for (int kk = 0; kk < kBN / 32; ++kk)
+  for (int kk = 0; kk < kSteps / 2; ++kk)
     if (ptx::elect_one())
-      ptx::mma_ts(tO, tP + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::kBoxBytes, 1024), kIdescPV,
-                  kk > 0 ? 1u : acc0);
-  if (!wait_warp(bar_p_full<D>(bar0, Q), s.pwait & 1u, c.abort_flag, p)) return false;
+      mma_ts_any<C>(tO, tP + kk * 8, smem_desc_sw128(vbase + kk * kVStep, C::kBoxBytes, 1024), kIdescPV,
+                    kk > 0 ? 1u : acc0);
+  if (!wait_warp(bar_p_full<C>(bar0, Q), s.pwait & 1u, c.abort_flag, p)) return false;
   ++s.pwait;
   ptx::tc_fence_after();
 #pragma unroll
-  for (int kk = kBN / 32; kk < kBN / 16; ++kk)
+  for (int kk = kSteps / 2; kk < kSteps; ++kk)
     if (ptx::elect_one())
-      ptx::mma_ts(tO, tP + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::kBoxBytes, 1024), kIdescPV,
-                  1u);
-  if (C::kSeparateP && ptx::elect_one()) ptx::mma_commit(bar_pv_done<D>(bar0, Q));
+      mma_ts_any<C>(tO, tP + kk * 8, smem_desc_sw128(vbase + kk * kVStep, C::kBoxBytes, 1024), kIdescPV,
+                    1u);
+  if (C::kSeparateP && ptx::elect_one()) ptx::mma_commit(bar_pv_done<C>(bar0, Q));
   ++s.npv;
   s.pend = -1;
   return true;
@@ -399,44 +440,45 @@ __device__ __forceinline__ bool mma_issue_pv(const MmaCtx<D>& c, const KernelPar
 
 // S_q = Q_q K_j^T into slot Q's S columns (warp-uniform).  With the
 // separate-P layout the softmax must first have read the previous S_q.
-template <int D, int Q>
-__device__ __forceinline__ bool mma_issue_s(const MmaCtx<D>& c, const KernelParams& p, MmaSlot& s,
+template <class C, int Q>
+__device__ __forceinline__ bool mma_issue_s(const MmaCtx<C>& c, const KernelParams& p, MmaSlot& s,
                                             int kslot, uint32_t bar0) {
-  using C = Cfg<D>;
-  constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
+  constexpr int D = C::kD;
+  constexpr uint32_t kIdescQK = C::kFp8 ? idesc_e4m3(128, 128, false) : idesc_bf16(128, 128, false);
   if (C::kSeparateP && s.ns > 0) {
-    if (!wait_warp(bar_s_free<D>(bar0, Q), (s.ns - 1) & 1u, c.abort_flag, p)) return false;
+    if (!wait_warp(bar_s_free<C>(bar0, Q), (s.ns - 1) & 1u, c.abort_flag, p)) return false;
     ptx::tc_fence_after();
   }
   const uint32_t qbase = c.sQ + Q * C::kTileBytes;
   const uint32_t kbase = c.sRing + kslot * C::kTileBytes;
   const uint32_t tS = c.tmem + (Q ? C::kTmemS1 : C::kTmemS0);
+  // Four K steps of 32 bytes per 128-byte box row.
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
+  for (int kk = 0; kk < D / C::kKStep; ++kk) {
     const uint32_t off = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
     if (ptx::elect_one())
-      ptx::mma_ss(tS, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                  kIdescQK, kk > 0 ? 1u : 0u);
+      mma_ss_any<C>(tS, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                    kIdescQK, kk > 0 ? 1u : 0u);
   }
-  if (ptx::elect_one()) ptx::mma_commit(bar_s_full<D>(bar0, Q));
+  if (ptx::elect_one()) ptx::mma_commit(bar_s_full<C>(bar0, Q));
   ++s.ns;
   return true;
 }
 
 // One kept K tile for slot Q in the P-over-S layout: settle its pending PV
 // (P_q shares columns with S_q), then S_q = Q_q K_j^T.  Warp-uniform.
-template <int D, int Q>
-__device__ __forceinline__ bool mma_slot_step(const MmaCtx<D>& c, const KernelParams& p, MmaSlot& s,
+template <class C, int Q>
+__device__ __forceinline__ bool mma_slot_step(const MmaCtx<C>& c, const KernelParams& p, MmaSlot& s,
                                               int64_t& v_ready, int kslot, uint32_t vr, uint32_t bar0) {
-  if (s.pend >= 0 && !mma_issue_pv<D, Q>(c, p, s, v_ready, bar0)) return false;
-  if (!mma_issue_s<D, Q>(c, p, s, kslot, bar0)) return false;
+  if (s.pend >= 0 && !mma_issue_pv<C, Q>(c, p, s, v_ready, bar0)) return false;
+  if (!mma_issue_s<C, Q>(c, p, s, kslot, bar0)) return false;
   s.pend = vr;
   return true;
 }
 
-template <int D, bool kVarlen = false>
+template <class C, bool kVarlen = false>
 __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_constant__ KernelParams p) {
-  using C = Cfg<D>;
+  constexpr int D = C::kD;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -446,14 +488,14 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   const uint32_t sRing = base + C::kOffRing;
   const uint32_t bar0 = base + C::kOffBar;
   const uint32_t bQFull = bar0, bQEmpty = bar0 + 8;
-  auto bFull = [&](int s) { return bar_full<D>(bar0, s); };
+  auto bFull = [&](int s) { return bar_full<C>(bar0, s); };
   auto bEmpty = [&](int s) { return bar0 + 16 + 8u * (C::kStages + s); };
-  auto bSFull = [&](int q) { return bar_s_full<D>(bar0, q); };
-  auto bPFull = [&](int q) { return bar_p_full<D>(bar0, q); };
-  auto bOFull = [&](int q) { return bar_o_full<D>(bar0, q); };
-  auto bOEmpty = [&](int q) { return bar_o_empty<D>(bar0, q); };
-  auto bPHalf = [&](int q) { return bar_p_half<D>(bar0, q); };
-  const uint32_t bMmaDone = bar_mma_done<D>(bar0);
+  auto bSFull = [&](int q) { return bar_s_full<C>(bar0, q); };
+  auto bPFull = [&](int q) { return bar_p_full<C>(bar0, q); };
+  auto bOFull = [&](int q) { return bar_o_full<C>(bar0, q); };
+  auto bOEmpty = [&](int q) { return bar_o_empty<C>(bar0, q); };
+  auto bPHalf = [&](int q) { return bar_p_half<C>(bar0, q); };
+  const uint32_t bMmaDone = bar_mma_done<C>(bar0);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kOffMisc + 4);
 
@@ -473,8 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       ptx::mbar_init(bOFull(q), 1);
       ptx::mbar_init(bOEmpty(q), 128);
       ptx::mbar_init(bPHalf(q), 128);
-      ptx::mbar_init(bar_s_free<D>(bar0, q), 128);
-      ptx::mbar_init(bar_pv_done<D>(bar0, q), 1);
+      ptx::mbar_init(bar_s_free<C>(bar0, q), 128);
+      ptx::mbar_init(bar_pv_done<C>(bar0, q), 1);
     }
     ptx::mbar_init(bMmaDone, 1);
     *abort_flag = 0;
@@ -515,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           int y, z;
           tile_coords<kVarlen>((qt0 + q) * kBM, bh, sq.h(), sq.q0(), y, z);
           for (int bx = 0; bx < C::kBoxes; ++bx)
-            ptx::tma_load_3d(sQ + q * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q, bQFull, bx * 64, y, z);
+            ptx::tma_load_3d(sQ + q * C::kTileBytes + bx * C::kBoxBytes, &p.tm_q, bQFull, bx * C::kBoxCols, y, z);
         }
       }
       ++nq;
@@ -537,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
                 tile_coords<kVarlen>(j * kBN, bh, sq.h(), sq.k0(), y, z);
                 for (int bx = 0; bx < C::kBoxes; ++bx)
                   ptx::tma_load_3d(sRing + slot * C::kTileBytes + bx * C::kBoxBytes, map,
-                                   bFull(slot), bx * 64, y, z);
+                                   bFull(slot), bx * C::kBoxCols, y, z);
               }
               ++it;
             }
@@ -558,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     uint32_t nq = 0;              // Q tiles consumed
     int64_t v_ready = -1;         // ring index of the newest V whose load was awaited
     bool ok = true;
-    const MmaCtx<D> ctx{tmem, sQ, sRing, abort_flag};
+    const MmaCtx<C> ctx{tmem, sQ, sRing, abort_flag};
     for (int w = blockIdx.x; w < p.items && ok; w += gridDim.x) {
       int bh, pair, split;
       decode_item(p, w, bh, pair, split);
@@ -590,23 +632,23 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           if constexpr (C::kSeparateP) {
             // Both S first (the softmax has already read the previous S), then
             // the PVs of the previous tile, whose P lives in its own columns.
-            if (ok && keep0) ok = mma_issue_s<D, 0>(ctx, p, slot0, kslot, bar0);
-            if (ok && keep1) ok = mma_issue_s<D, 1>(ctx, p, slot1, kslot, bar0);
+            if (ok && keep0) ok = mma_issue_s<C, 0>(ctx, p, slot0, kslot, bar0);
+            if (ok && keep1) ok = mma_issue_s<C, 1>(ctx, p, slot1, kslot, bar0);
             if (ok && ptx::elect_one()) ptx::mma_commit(bEmpty(kslot));  // K_j no longer needed
-            if (ok && slot0.pend >= 0) ok = mma_issue_pv<D, 0>(ctx, p, slot0, v_ready, bar0);
-            if (ok && slot1.pend >= 0) ok = mma_issue_pv<D, 1>(ctx, p, slot1, v_ready, bar0);
+            if (ok && slot0.pend >= 0) ok = mma_issue_pv<C, 0>(ctx, p, slot0, v_ready, bar0);
+            if (ok && slot1.pend >= 0) ok = mma_issue_pv<C, 1>(ctx, p, slot1, v_ready, bar0);
             if (keep0) slot0.pend = vr;
             if (keep1) slot1.pend = vr;
           } else {
             // Slot q: pending O_q += P_q V first (P_q shares columns with S_q),
             // then S_q = Q_q K_j^T.
-            if (ok && keep0) ok = mma_slot_step<D, 0>(ctx, p, slot0, v_ready, kslot, vr, bar0);
-            if (ok && keep1) ok = mma_slot_step<D, 1>(ctx, p, slot1, v_ready, kslot, vr, bar0);
+            if (ok && keep0) ok = mma_slot_step<C, 0>(ctx, p, slot0, v_ready, kslot, vr, bar0);
+            if (ok && keep1) ok = mma_slot_step<C, 1>(ctx, p, slot1, v_ready, kslot, vr, bar0);
             if (ok && ptx::elect_one()) ptx::mma_commit(bEmpty(kslot));  // K_j no longer needed
             // A slot that skips K_j still owes a PV on the previous V: issue it
             // now so that V can be released.
-            if (ok && !keep0 && slot0.pend >= 0) ok = mma_issue_pv<D, 0>(ctx, p, slot0, v_ready, bar0);
-            if (ok && !keep1 && slot1.pend >= 0) ok = mma_issue_pv<D, 1>(ctx, p, slot1, v_ready, bar0);
+            if (ok && !keep0 && slot0.pend >= 0) ok = mma_issue_pv<C, 0>(ctx, p, slot0, v_ready, bar0);
+            if (ok && !keep1 && slot1.pend >= 0) ok = mma_issue_pv<C, 1>(ctx, p, slot1, v_ready, bar0);
           }
           if (ok && prev_v >= 0 && ptx::elect_one())
             ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
@@ -616,13 +658,13 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       if (ok) {
         // Every S MMA of this unit is issued: Q may be replaced once they finish.
         if (ptx::elect_one()) ptx::mma_commit(bQEmpty);
-        if (slot0.pend >= 0) ok = mma_issue_pv<D, 0>(ctx, p, slot0, v_ready, bar0);
-        if (ok && slot1.pend >= 0) ok = mma_issue_pv<D, 1>(ctx, p, slot1, v_ready, bar0);
+        if (slot0.pend >= 0) ok = mma_issue_pv<C, 0>(ctx, p, slot0, v_ready, bar0);
+        if (ok && slot1.pend >= 0) ok = mma_issue_pv<C, 1>(ctx, p, slot1, v_ready, bar0);
         if (ok && prev_v >= 0 && ptx::elect_one())
           ptx::mma_commit(bEmpty((int)(prev_v % C::kStages)));
         if (ok && ptx::elect_one()) {
-          if (slot0.npv > 0) ptx::mma_commit(bar_o_full<D>(bar0, 0));
-          if (valid1 && slot1.npv > 0) ptx::mma_commit(bar_o_full<D>(bar0, 1));
+          if (slot0.npv > 0) ptx::mma_commit(bar_o_full<C>(bar0, 0));
+          if (valid1 && slot1.npv > 0) ptx::mma_commit(bar_o_full<C>(bar0, 1));
         }
       }
       slot0.end_unit(true);
@@ -671,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           ptx::tmem_wait_ld();
           if constexpr (C::kSeparateP) {  // S_q may now be overwritten by the next tile
             ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_s_free<D>(bar0, q));
+            ptx::mbar_arrive(bar_s_free<C>(bar0, q));
           }
           float s[128];
 #pragma unroll
@@ -700,18 +742,18 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           const float m_new = fmaxf(m_ref, tmax * sl);
           // Move the reference max only when the new one exceeds it by more than
           // 2^kRescaleLog2 (always on the first visible tile: m_ref = -inf).
-          const bool rescale = m_new > m_ref + kRescaleLog2;
+          const bool rescale = m_new > m_ref + C::kRescale;
           float alpha = 1.f;
           if (rescale) {
             alpha = ptx::ex2(m_ref - m_new);  // 0 when m_ref = -inf
             l *= alpha;
             m_ref = m_new;
           }
-          const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          const float neg_m = (m_ref == -INFINITY) ? 0.f : C::kPShift - m_ref;
           if constexpr (C::kSeparateP) {
             // P_q and O_q are still read / written by the previous tile's PV.
             if (swait >= 2) {
-              ok = wait_warp(bar_pv_done<D>(bar0, q), (swait - 2) & 1u, abort_flag, p);
+              ok = wait_warp(bar_pv_done<C>(bar0, q), (swait - 2) & 1u, abort_flag, p);
               if (!ok) break;
               ptx::tc_fence_after();
             }
@@ -722,7 +764,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           // exponentials of the second.
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            uint32_t pk[32];
+            // P of keys [64 half, 64 half + 64): 32 words of two bf16, or 16
+            // words of four e4m3; l sums exactly the rounded values.
+            uint32_t pk[C::kFp8 ? 16 : 32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               const int cc = 32 * half + c;
@@ -734,11 +778,23 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
                 p0 = ptx::ex2(x0);
                 p1 = ptx::ex2(x1);
               }
-              const uint32_t w2 = ptx::pack_bf16x2(p0, p1);
-              pk[c] = w2;
-              ptx::add_bf16x2(ls[2 * (c & 1)], ls[2 * (c & 1) + 1], w2);
+              if constexpr (C::kFp8) {
+                if (c & 1) {
+                  const uint32_t w4 = ptx::pack_e4m3x4(s[2 * cc - 2], s[2 * cc - 1], p0, p1);
+                  pk[c >> 1] = w4;
+                  ptx::add_e4m3x4(ls[2 * ((c >> 1) & 1)], ls[2 * ((c >> 1) & 1) + 1], w4);
+                } else {
+                  s[2 * cc] = p0;  // held until the next pair completes the word
+                  s[2 * cc + 1] = p1;
+                }
+              } else {
+                const uint32_t w2 = ptx::pack_bf16x2(p0, p1);
+                pk[c] = w2;
+                ptx::add_bf16x2(ls[2 * (c & 1)], ls[2 * (c & 1) + 1], w2);
+              }
             }
-            ptx::tmem_st32(tP + 32 * half, pk);
+            if constexpr (C::kFp8) ptx::tmem_st16(tP + 16 * half, pk);
+            else ptx::tmem_st32(tP + 32 * half, pk);
             if (half == 0) {
               // O holds earlier tiles: rescale it in place before any PV of this
               // tile.  tcgen05.ld/st are warp-collective, so the warp rescales
@@ -777,7 +833,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       // A row whose reference max never left -inf saw no visible key (masked
       // scores only add 2^-125 through the FMA-pipe exp2): O = 0, lse = -inf.
       const bool seen = m_ref != -INFINITY && l > 0.f;
-      const float inv = seen ? 1.f / l : 0.f;
+      const float inv = seen ? p.o_scale / l : 0.f;
+      const float lse2 = m_ref - C::kPShift + log2f(l);  // log2 of the row's sum, scaled scores
       // Sizes again (not held in registers across the tile loop).
       const auto se = seq_of<kVarlen>(p, bh);
       const bool in_range = row < se.nq();
@@ -803,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           }
         }
         if (in_range)
-          p.part_lse[prow] = seen ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+          p.part_lse[prow] = seen ? lse2 * 0.69314718055994530942f : -INFINITY;
       } else {
       // O row and lse element of this query: [B*H][Nq] rows, or token-major
       // [T][H] rows with lse [H][T] for variable-length batches.
@@ -832,7 +889,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
         }
       }
       if (in_range)
-        p.lse[lse_i] = seen ? (m_ref + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        p.lse[lse_i] = seen ? lse2 * 0.69314718055994530942f : -INFINITY;
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(bOEmpty(q));

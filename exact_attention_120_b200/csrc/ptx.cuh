@@ -148,6 +148,28 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// The same two forms for kind::f8f6f4 (8-bit operands, formats in the
+// instruction descriptor; K = 32 per instruction).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile(
@@ -258,6 +280,36 @@ __device__ __forceinline__ void add_bf16x2(float& acc_lo, float& acc_hi, uint32_
       "mov.b32 {lo, hi}, %2;\n\t"
       "add.rn.f32.bf16 %0, lo, %0;\n\t"
       "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc_lo), "+f"(acc_hi)
+      : "r"(w));
+}
+
+// Four floats -> four e4m3 bytes (round to nearest even, saturating to
+// +-448), x0 in bits [0, 8) ... x3 in bits [24, 32).
+__device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, float x3) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
+  return r;
+}
+
+// acc_lo += bytes 0 and 2 of w, acc_hi += bytes 1 and 3 (four e4m3 values,
+// widened exactly to f16, each added in fp32 with one rounding).
+__device__ __forceinline__ void add_e4m3x4(float& acc_lo, float& acc_hi, uint32_t w) {
+  asm("{\n\t.reg .b16 e0, e1, h0, h1, h2, h3;\n\t.reg .b32 f0, f1;\n\t"
+      "mov.b32 {e0, e1}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 f0, e0;\n\t"
+      "cvt.rn.f16x2.e4m3x2 f1, e1;\n\t"
+      "mov.b32 {h0, h1}, f0;\n\t"
+      "mov.b32 {h2, h3}, f1;\n\t"
+      "add.rn.f32.f16 %0, h0, %0;\n\t"
+      "add.rn.f32.f16 %1, h1, %1;\n\t"
+      "add.rn.f32.f16 %0, h2, %0;\n\t"
+      "add.rn.f32.f16 %1, h3, %1;\n\t}"
       : "+f"(acc_lo), "+f"(acc_hi)
       : "r"(w));
 }

@@ -186,3 +186,27 @@ def varlen_flops(lengths_q, lengths_k, H, d, causal):
             vis = nq * nk
         f += 4.0 * d * H * vis
     return f
+
+
+# ------------------------------------------------------------------ fp8 ---
+# 8-bit inputs: the same float32 draws as make_qkv, each tensor quantised to
+# OCP E4M3 with one scale per tensor (amax / 448, so the largest magnitude
+# maps to the format's largest finite value), rounding by PyTorch's
+# float8_e4m3fn conversion.  Quantisation is the caller's step, not part of
+# the attention being computed.
+
+
+def make_qkv_fp8(B, H, N, d, seed, qk_std=1.0, v_std=1.0, Nk=None):
+    """(q8, k8, v8) uint8 codes [B, H, N(k), d] on the CPU and their
+    dequantisation scales (q_descale, k_descale, v_descale)."""
+    Nk = N if Nk is None else Nk
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    xs = [torch.randn((B, H, N, d), generator=g) * qk_std,
+          torch.randn((B, H, Nk, d), generator=g) * qk_std,
+          torch.randn((B, H, Nk, d), generator=g) * v_std]
+    codes, scales = [], []
+    for x in xs:
+        s = float(x.abs().max()) / 448.0
+        codes.append((x / s).to(torch.float8_e4m3fn).view(torch.uint8).contiguous())
+        scales.append(s)
+    return tuple(codes), tuple(scales)

@@ -168,6 +168,32 @@ FA_API int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, v
 FA_API int fa_fwd_splitkv_heuristic(int B, int H, int Nq, int Nk);
 
 /*
+ * 8-bit forward: the same attention on FP8 (e4m3) inputs, the low-precision
+ * direction the pages name for the next FlashAttention generation
+ * (wmrh.cn article, section "FlashAttention 的局限和后续发展").  q, k, v hold
+ * e4m3 codes (OCP FP8 E4M3: bias 7, no infinities, largest finite 448)
+ * standing for q_descale * q, k_descale * k, v_descale * v; the result is the
+ * attention of those real values, exactly as fa_fwd_qk defines it:
+ *   O = softmax(scale * (q_descale q)(k_descale k)^T) (v_descale v).
+ * Both products run on the 8-bit tensor-core path (kind::f8f6f4) with fp32
+ * accumulation; P is rounded to e4m3 before the PV product and the row sums
+ * add those same rounded values, so every O row is an exact weighted mean of
+ * V rows with each weight off by at most 2^-4 relative.
+ *
+ * q: [B, H, Nq, d]; k, v: [B, H, Nk, d], one byte per element, contiguous,
+ * 16-byte aligned; o: bf16 [B, H, Nq, d]; lse: fp32 [B, H, Nq] (natural log
+ * of the scaled scores, as fa_fwd).  d must be 128.  causal and block_mask as
+ * in fa_fwd_qk.  Descales finite and > 0.  Asynchronous on cuda_stream.
+ *
+ * Returns FA_OK, FA_ERR_INVALID_ARGUMENT (as fa_fwd_qk, or a bad descale),
+ * FA_ERR_UNSUPPORTED (d != 128, sizes as fa_fwd_qk) or FA_ERR_CUDA.
+ */
+FA_API int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int Nq, int Nk, int d, float scale, int causal,
+                      const uint8_t* block_mask, float q_descale, float k_descale,
+                      float v_descale, void* cuda_stream);
+
+/*
  * Variable-length batch: B independent attention problems of different
  * lengths in one launch, the layout of packed token streams.  Sequence b
  * owns query token rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key/value
