@@ -73,16 +73,16 @@ int setup_device(int dev, DeviceState& st) {
     e = cudaFuncSetAttribute(fa::fa_fwd_kernel<fa::Cfg<128>, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::Cfg<128>::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(fa::fa_bwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            fa::BwdCfg<64>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(fa::fa_bwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::BwdCfg<128>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(fa::fa_bwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::BwdCfg<64>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(fa::fa_bwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fa::BwdCfg<128>::kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e);
   void* sym = nullptr;
@@ -431,18 +431,18 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   p.causal = causal;
   p.scale = scale;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
-    p.timeout_ns = kWaitTimeoutNs;
+  p.timeout_ns = kWaitTimeoutNs;
   p.status = st->status_word;
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int grid_q = (int)std::min<long long>(bh * nqt, st->num_sms);
   const int grid_k = (int)std::min<long long>(bh * nkt, st->num_sms);
   if (d == 64) {
-    fa::fa_bwd_dq_kernel<64><<<grid_q, fa::kBwdThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(p);
-    fa::fa_bwd_dkdv_kernel<64><<<grid_k, fa::kBwdThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(p);
+    fa::fa_bwd_kernel<64, true><<<grid_q, fa::kBwdThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(p);
+    fa::fa_bwd_kernel<64, false><<<grid_k, fa::kBwdThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(p);
   } else {
-    fa::fa_bwd_dq_kernel<128><<<grid_q, fa::kBwdThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(p);
-    fa::fa_bwd_dkdv_kernel<128><<<grid_k, fa::kBwdThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(p);
+    fa::fa_bwd_kernel<128, true><<<grid_q, fa::kBwdThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(p);
+    fa::fa_bwd_kernel<128, false><<<grid_k, fa::kBwdThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(p);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
