@@ -168,6 +168,14 @@ int encode_varlen_map(CUtensorMap* map, const void* ptr, int T, int H, int d) {
 
 constexpr int kMaxSplits = 256;
 
+// Heads per group of the causal work order: as many as keep their K and V
+// (2 x nk x d x elt_bytes each) within ~96 MB of the 126 MB L2.
+int causal_group(long long bh, long long nk, int d, int elt_bytes) {
+  const long long kv = 2ll * std::max(nk, 1ll) * d * elt_bytes;
+  const long long g = (96ll << 20) / kv;
+  return (int)std::max(1ll, std::min(bh, g));
+}
+
 // Workspace of fa_fwd_splitkv_noalloc: a fixed array in the module's device
 // memory, so that entry point never allocates.  Every device that loads the
 // library holds it until the process exits; all calls on a device share it.
@@ -255,6 +263,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.causal_off = Nk - Nq;
   p.npairs = (int)npairs;
   p.bh = (int)bh;
+  p.group = causal_group(bh, Nk, d, eb);
   p.items = (int)(bh * npairs * splits);
   p.splits = splits;
   p.kt_per_split = kt_per_split;
@@ -505,6 +514,9 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   p.causal_off = 0;
   p.npairs = (int)npairs;
   p.bh = (int)bh;
+  // Sequences are at most max_seqlen_q long; keys of the longest are bounded
+  // by total_k, so group by the query bound (the usual self-attention case).
+  p.group = causal_group(bh, std::min<long long>(max_seqlen_q, total_k), d, 2);
   p.items = (int)(bh * npairs);
   p.splits = 1;
   p.kt_per_split = p.nkt;

@@ -438,48 +438,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           int last = p.Nk - 1;
           if (p.causal) last = min(last, row + p.causal_off);
           const int lim = last - col0;
-#pragma unroll 1
-          for (int ch = 0; ch < 2; ++ch) {
-            uint32_t rs[32], rp[32];
-            ptx::tmem_ld32(tS + 32 * ch, rs);
-            ptx::tmem_ld32(tG + 32 * ch, rp);
-            ptx::tmem_wait_ld();
-            uint32_t pk[16];
+          // All 64 scores and 64 gradients in one round trip.
+          uint32_t rs[2][32], rp[2][32];
+          ptx::tmem_ld32(tS, rs[0]);
+          ptx::tmem_ld32(tS + 32, rs[1]);
+          ptx::tmem_ld32(tG, rp[0]);
+          ptx::tmem_ld32(tG + 32, rp[1]);
+          ptx::tmem_wait_ld();
+          uint32_t pk[32];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float ds[2];
+          for (int e = 0; e < 32; ++e) {
+            float ds[2];
 #pragma unroll
-              for (int k = 0; k < 2; ++k) {
-                const int col = 32 * ch + 2 * e + k;
-                const float pr = col <= lim ? ptx::ex2(fmaf(__uint_as_float(rs[2 * e + k]), c, nlse2)) : 0.f;
-                ds[k] = pr * (__uint_as_float(rp[2 * e + k]) - delta);
-              }
-              pk[e] = ptx::pack_bf16x2(ds[0], ds[1]);
+            for (int k = 0; k < 2; ++k) {
+              const int col = 2 * e + k;
+              const float pr = col <= lim ? ptx::ex2(fmaf(__uint_as_float(rs[col >> 5][col & 31]), c, nlse2)) : 0.f;
+              ds[k] = pr * (__uint_as_float(rp[col >> 5][col & 31]) - delta);
             }
-            // dS over S columns [16 ch, 16 ch + 16): already read.
-            ptx::tmem_st16(tS + 16 * ch, pk);
+            pk[e] = ptx::pack_bf16x2(ds[0], ds[1]);
           }
+          ptx::tmem_st32(tS, pk);  // dS over S columns [0, 32)
         } else {
           // Visible queries of this key row within the half: c >= lo.
           const int lo = p.causal ? row - p.causal_off - col0 : INT_MIN;
           const float* v = vals + (it % C::kStages) * 256 + 64 * h;
-#pragma unroll 1
+          uint32_t rs[2][32], rp[2][32];
+          ptx::tmem_ld32(tS, rs[0]);
+          ptx::tmem_ld32(tS + 32, rs[1]);
+          ptx::tmem_ld32(tG, rp[0]);
+          ptx::tmem_ld32(tG + 32, rp[1]);
+          ptx::tmem_wait_ld();
+          // P^T over S^T columns [16 ch, 16 ch + 16), dS^T likewise over dP^T.
+#pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
-            uint32_t rs[32], rp[32];
-            ptx::tmem_ld32(tS + 32 * ch, rs);
-            ptx::tmem_ld32(tG + 32 * ch, rp);
-            ptx::tmem_wait_ld();
             uint32_t pp[16], pd[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const int col = 32 * ch + 2 * e;
+              const int k = 2 * e;
+              const int col = 32 * ch + k;
               const float2 nl = *reinterpret_cast<const float2*>(v + col);
               const float2 dl = *reinterpret_cast<const float2*>(v + 128 + col);
-              const float p0 = col >= lo ? ptx::ex2(fmaf(__uint_as_float(rs[2 * e]), c, nl.x)) : 0.f;
-              const float p1 = col + 1 >= lo ? ptx::ex2(fmaf(__uint_as_float(rs[2 * e + 1]), c, nl.y)) : 0.f;
+              const float p0 = col >= lo ? ptx::ex2(fmaf(__uint_as_float(rs[ch][k]), c, nl.x)) : 0.f;
+              const float p1 = col + 1 >= lo ? ptx::ex2(fmaf(__uint_as_float(rs[ch][k + 1]), c, nl.y)) : 0.f;
               pp[e] = ptx::pack_bf16x2(p0, p1);
-              pd[e] = ptx::pack_bf16x2(p0 * (__uint_as_float(rp[2 * e]) - dl.x),
-                                       p1 * (__uint_as_float(rp[2 * e + 1]) - dl.y));
+              pd[e] = ptx::pack_bf16x2(p0 * (__uint_as_float(rp[ch][k]) - dl.x),
+                                       p1 * (__uint_as_float(rp[ch][k + 1]) - dl.y));
             }
             ptx::tmem_st16(tS + 16 * ch, pp);
             ptx::tmem_st16(tG + 16 * ch, pd);

@@ -74,6 +74,7 @@ struct KernelParams {
   int causal_off;  // Nk - Nq: key j is visible to query i iff j <= i + causal_off
   int npairs;      // work units per head
   int bh;      // B * H
+  int group;   // causal order: heads per group (their K/V together fit in L2)
   int items;   // bh * npairs
   int causal;
   float scale_log2;  // scale * log2(e) (8-bit inputs: times the Q and K dequantisation scales)
@@ -271,9 +272,15 @@ __device__ __forceinline__ void decode_item(const KernelParams& p, int w, int& b
                                             int& split) {
   split = w % p.splits;  // the slices of one unit run side by side
   w /= p.splits;
-  if (p.causal) {  // longest rows first, all heads interleaved
-    pair = p.npairs - 1 - w / p.bh;
-    bh = w % p.bh;
+  if (p.causal) {
+    // Longest rows first, heads interleaved within groups of p.group heads
+    // whose K/V fit in L2 together (one group when all heads fit).
+    const int per_group = p.group * p.npairs;
+    const int g = w / per_group;
+    const int r = w - g * per_group;
+    const int gsz = min(p.group, p.bh - g * p.group);
+    pair = p.npairs - 1 - r / gsz;
+    bh = g * p.group + r % gsz;
   } else {  // all pairs of one head together: that head's K/V stays in L2
     bh = w / p.npairs;
     pair = w % p.npairs;
