@@ -28,6 +28,8 @@
 // records FA_ERR_DEVICE_TIMEOUT, leaves its loops, drains and frees TMEM.
 #pragma once
 
+#include <type_traits>
+
 #include "fa_fwd_kernel.cuh"
 
 namespace fa {
@@ -64,7 +66,7 @@ struct BwdCfg {
   static constexpr int kStages = (D == 128) ? 2 : 4;  // streamed tile pairs in flight
   // Shared memory: stationary tiles A, B (kDQ: Q, dO; else K, V), the ring of
   // streamed pairs X, Y (kDQ: K_j, V_j; else Q_i, dO_i), and for the dK/dV
-  // launch the column values of each ring slot (-log2(e) lse_q, D_q).
+  // launch the column values of each ring slot (-log2(e) lse_q, -D_q).
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kTileBytes;
   static constexpr int kOffRing = 2 * kTileBytes;
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
         }
         if constexpr (!kDQ) {
           // Column values of query tile x: -log2(e) lse_q (-inf past Nq or
-          // for a query without keys, so its P is 0) and D_q.
+          // for a query without keys, so its P is 0) and -D_q.
           float* v = vals + s * 256;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
               dd = p.delta[(size_t)u.bh * p.Nq + q];
             }
             v[c] = (l == -INFINITY) ? -INFINITY : -l * kLog2e;
-            v[128 + c] = dd;
+            v[128 + c] = -dd;
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(bars.full(s));
@@ -426,6 +428,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           if (h == 0) p.delta[(size_t)u.bh * p.Nq + row] = delta;
         }
       }
+      const float ndelta = -delta;
       int ntiles = 0;
       for (int x = u.next(p, -1); x < u.end(p) && ok; x = u.next(p, x)) {
         ok = bwd_wait(bars.s_full(h), sw & 1u, abort_flag, p);
@@ -446,44 +449,76 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
           ptx::tmem_ld32(tG + 32, rp[1]);
           ptx::tmem_wait_ld();
           uint32_t pk[32];
+          // Pairs of columns with packed f32x2 arithmetic; the mask only on
+          // tiles that reach the diagonal or the end of the keys.
+          auto body = [&](auto masked) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float ds[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int col = 2 * e + k;
-              const float pr = col <= lim ? ptx::ex2(fmaf(__uint_as_float(rs[col >> 5][col & 31]), c, nlse2)) : 0.f;
-              ds[k] = pr * (__uint_as_float(rp[col >> 5][col & 31]) - delta);
+            for (int e = 0; e < 32; ++e) {
+              const int col = 2 * e;
+              float x0, x1, p0, p1, g0, g1, d0, d1;
+              ptx::fma2(x0, x1, __uint_as_float(rs[col >> 5][col & 31]),
+                        __uint_as_float(rs[col >> 5][(col & 31) + 1]), c, c, nlse2, nlse2);
+              p0 = ptx::ex2(x0);
+              p1 = ptx::ex2(x1);
+              if constexpr (decltype(masked)::value) {
+                p0 = col <= lim ? p0 : 0.f;
+                p1 = col + 1 <= lim ? p1 : 0.f;
+              }
+              ptx::add2(g0, g1, __uint_as_float(rp[col >> 5][col & 31]),
+                        __uint_as_float(rp[col >> 5][(col & 31) + 1]), ndelta, ndelta);
+              ptx::mul2(d0, d1, p0, p1, g0, g1);
+              pk[e] = ptx::pack_bf16x2(d0, d1);
             }
-            pk[e] = ptx::pack_bf16x2(ds[0], ds[1]);
-          }
+          };
+          if (__all_sync(0xffffffffu, lim >= 63)) body(std::false_type{});
+          else body(std::true_type{});
           ptx::tmem_st32(tS, pk);  // dS over S columns [0, 32)
         } else {
           // Visible queries of this key row within the half: c >= lo.
           const int lo = p.causal ? row - p.causal_off - col0 : INT_MIN;
           const float* v = vals + (it % C::kStages) * 256 + 64 * h;
-          uint32_t rs[2][32], rp[2][32];
-          ptx::tmem_ld32(tS, rs[0]);
-          ptx::tmem_ld32(tS + 32, rs[1]);
-          ptx::tmem_ld32(tG, rp[0]);
-          ptx::tmem_ld32(tG + 32, rp[1]);
-          ptx::tmem_wait_ld();
-          // P^T over S^T columns [16 ch, 16 ch + 16), dS^T likewise over dP^T.
-#pragma unroll
+          // 32 columns at a time: P^T over S^T columns [16 ch, 16 ch + 16),
+          // dS^T likewise over dP^T (both already read).  Four columns per
+          // step: their -log2(e) lse and -D as float4 (broadcast shared-memory
+          // reads), packed f32x2 arithmetic; the mask only on tiles that reach
+          // the causal diagonal.
+          const bool masked = !__all_sync(0xffffffffu, lo <= 0);
+#pragma unroll 1
           for (int ch = 0; ch < 2; ++ch) {
+            uint32_t rs[32], rp[32];
+            ptx::tmem_ld32(tS + 32 * ch, rs);
+            ptx::tmem_ld32(tG + 32 * ch, rp);
+            ptx::tmem_wait_ld();
             uint32_t pp[16], pd[16];
+            auto body = [&](auto mtag) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int k = 2 * e;
-              const int col = 32 * ch + k;
-              const float2 nl = *reinterpret_cast<const float2*>(v + col);
-              const float2 dl = *reinterpret_cast<const float2*>(v + 128 + col);
-              const float p0 = col >= lo ? ptx::ex2(fmaf(__uint_as_float(rs[ch][k]), c, nl.x)) : 0.f;
-              const float p1 = col + 1 >= lo ? ptx::ex2(fmaf(__uint_as_float(rs[ch][k + 1]), c, nl.y)) : 0.f;
-              pp[e] = ptx::pack_bf16x2(p0, p1);
-              pd[e] = ptx::pack_bf16x2(p0 * (__uint_as_float(rp[ch][k]) - dl.x),
-                                       p1 * (__uint_as_float(rp[ch][k + 1]) - dl.y));
-            }
+              for (int e4 = 0; e4 < 8; ++e4) {
+                const int k = 4 * e4;
+                const int col = 32 * ch + k;
+                const float4 nl = *reinterpret_cast<const float4*>(v + col);
+                const float4 nd = *reinterpret_cast<const float4*>(v + 128 + col);
+                const float nla[4] = {nl.x, nl.y, nl.z, nl.w}, nda[4] = {nd.x, nd.y, nd.z, nd.w};
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  float x0, x1, p0, p1, g0, g1, d0, d1;
+                  ptx::fma2(x0, x1, __uint_as_float(rs[k + 2 * j]), __uint_as_float(rs[k + 2 * j + 1]), c, c,
+                            nla[2 * j], nla[2 * j + 1]);
+                  p0 = ptx::ex2(x0);
+                  p1 = ptx::ex2(x1);
+                  if constexpr (decltype(mtag)::value) {
+                    p0 = col + 2 * j >= lo ? p0 : 0.f;
+                    p1 = col + 2 * j + 1 >= lo ? p1 : 0.f;
+                  }
+                  ptx::add2(g0, g1, __uint_as_float(rp[k + 2 * j]), __uint_as_float(rp[k + 2 * j + 1]),
+                            nda[2 * j], nda[2 * j + 1]);
+                  ptx::mul2(d0, d1, p0, p1, g0, g1);
+                  pp[2 * e4 + j] = ptx::pack_bf16x2(p0, p1);
+                  pd[2 * e4 + j] = ptx::pack_bf16x2(d0, d1);
+                }
+              }
+            };
+            if (masked) body(std::true_type{});
+            else body(std::false_type{});
             ptx::tmem_st16(tS + 16 * ch, pp);
             ptx::tmem_st16(tG + 16 * ch, pd);
           }
