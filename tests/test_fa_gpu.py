@@ -50,15 +50,32 @@ def test_wide_score_range_rescales():
     full_parity(q, k, v)
 
 
-def test_increasing_scores_force_rescale_every_tile():
+@pytest.mark.parametrize("d", [64, 128])
+def test_increasing_scores_force_rescale_every_tile(d):
     # Key norms grow along the sequence, so every new tile raises the max.
-    B, H, N, d = 1, 2, 1024, 64
+    B, H, N = 1, 2, 1024
     q, k, v, _ = make_case(B, H, N, d, seed=12)
     ramp = torch.linspace(0.2, 6.0, N).view(1, 1, N, 1)
     k = (k.float() * ramp).to(torch.bfloat16)
     q = (q.float().abs() + 0.5).to(torch.bfloat16)
     k = k.float().abs().to(torch.bfloat16)
     full_parity(q, k, v)
+
+
+@pytest.mark.parametrize("jump", [31.0, 80.0])
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_max_jump_within_a_unit(jump, causal):
+    # Keys of tile 3 score `jump` (log2 units) above everything before them:
+    # 31 moves the reference after the tile (its P reaches 2^31), 80 exceeds
+    # what one tile may absorb against the old reference and is redone.
+    B, H, N, d = 1, 2, 896, 128
+    q, k, v, _ = make_case(B, H, N, d, seed=21)
+    scale = 1 / math.sqrt(d)
+    q = torch.full((B, H, N, d), 8.0).to(torch.bfloat16)
+    k = (k.float() * 0.1).to(torch.bfloat16)
+    kval = jump / (math.log2(math.e) * scale * 8.0 * d)
+    k[:, :, 3 * 128:3 * 128 + 5] = kval
+    full_parity(q, k, v, causal=causal)
 
 
 def test_empty_rows_and_empty_tiles():
