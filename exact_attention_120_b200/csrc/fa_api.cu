@@ -423,6 +423,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if ((rc = encode_qkv_map(&p.tm_k, k, (int)bh, Nk, d)) != FA_OK) return rc;
   if ((rc = encode_qkv_map(&p.tm_v, v, (int)bh, Nk, d)) != FA_OK) return rc;
   if ((rc = encode_qkv_map(&p.tm_do, dout, (int)bh, Nq, d)) != FA_OK) return rc;
+  p.q = static_cast<const __nv_bfloat16*>(q);
   p.o = static_cast<const __nv_bfloat16*>(o);
   p.dout = static_cast<const __nv_bfloat16*>(dout);
   p.lse = lse;

@@ -39,6 +39,7 @@ struct BwdParams {
   CUtensorMap tm_k;   // [B*H][Nk][D]
   CUtensorMap tm_v;   // [B*H][Nk][D]
   CUtensorMap tm_do;  // [B*H][Nq][D]
+  const __nv_bfloat16* q;
   const __nv_bfloat16* o;
   const __nv_bfloat16* dout;
   const float* lse;  // [B*H][Nq]
@@ -81,8 +82,13 @@ struct BwdCfg {
   // (dP or dP^T) at [128h + 64, 128h + 128); the bf16 results are written
   // over the first 32 columns of each.  Accumulators: kDQ: dQ at [256, 256 + D);
   // else dV at [256, 256 + D) and dK at [256 + D, 256 + 2D).
+  // The dQ launch also keeps Q and dO in tensor memory ([256 + D, 256 + 3D/2)
+  // and [256 + 3D/2, 256 + 2D), bf16 pairs per column) as the A operands of S
+  // and dP: then the 64-wide score MMAs read only K and V from shared memory.
   static constexpr uint32_t kAcc0 = 256;
   static constexpr uint32_t kAcc1 = 256 + D;
+  static constexpr uint32_t kTq = 256 + D;
+  static constexpr uint32_t kTdo = 256 + D + D / 2;
   __host__ __device__ static constexpr uint32_t s_col(int h) { return 128u * h; }
   __host__ __device__ static constexpr uint32_t g_col(int h) { return 128u * h + 64u; }
 };
@@ -177,6 +183,18 @@ __device__ __forceinline__ void bwd_mma_half(uint32_t dtm, uint32_t a, uint32_t 
   }
 }
 
+// The same with A (128 x D bf16, D/2 columns) in tensor memory.
+template <int D>
+__device__ __forceinline__ void bwd_mma_half_ts(uint32_t dtm, uint32_t atm, uint32_t b_half) {
+  constexpr uint32_t kIdesc = idesc_bf16(128, 64, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * BwdCfg<D>::kBoxBytes + (kk & 3) * 32;
+    if (ptx::elect_one())
+      ptx::mma_ts(dtm, atm + kk * 8, smem_desc_sw128(b_half + off, 16, 1024), kIdesc, kk > 0 ? 1u : 0u);
+  }
+}
+
 // C[tmem, 128 x D] (+)= A[tmem, 128 x 64 bf16 (32 columns)] * B[smem, rows
 // 64h.. + 64 of a tile, used MN-major]: four K steps of 16 rows (2 KB).
 template <int D>
@@ -214,7 +232,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   const int items = p.bh * (kDQ ? p.nqt : p.nkt);
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bars.ab_full(), 1);
+    // dQ: both elementwise warpgroups arrive once Q and dO are in tensor
+    // memory; dK/dV: the producer's expect-tx arrival for the K, V tiles.
+    ptx::mbar_init(bars.ab_full(), kDQ ? 256 : 1);
     ptx::mbar_init(bars.ab_empty(), 1);
     for (int s = 0; s < C::kStages; ++s) {
       // dK/dV: the producer's expect-tx arrival plus one after it stored the
@@ -259,15 +279,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     bool ok = true;
     for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
       const BwdUnit<kDQ> u(p, w);
-      ok = bwd_wait(bars.ab_empty(), (nu & 1u) ^ 1u, abort_flag, p);
-      if (!ok) break;
-      if (ptx::elect_one()) {
-        ptx::mbar_arrive_expect_tx(bars.ab_full(), 2 * C::kTileBytes);
-        bwd_load_tile<D>(sA, mapA, bars.ab_full(), u.t * kBM, u.bh);
-        bwd_load_tile<D>(sB, mapB, bars.ab_full(), u.t * kBM, u.bh);
+      if constexpr (!kDQ) {
+        ok = bwd_wait(bars.ab_empty(), (nu & 1u) ^ 1u, abort_flag, p);
+        if (!ok) break;
+        if (ptx::elect_one()) {
+          ptx::mbar_arrive_expect_tx(bars.ab_full(), 2 * C::kTileBytes);
+          bwd_load_tile<D>(sA, mapA, bars.ab_full(), u.t * kBM, u.bh);
+          bwd_load_tile<D>(sB, mapB, bars.ab_full(), u.t * kBM, u.bh);
+        }
+        __syncwarp();
+        ++nu;
       }
-      __syncwarp();
-      ++nu;
       for (int x = u.next(p, -1); x < u.end(p) && ok; x = u.next(p, x)) {
         const int s = it % C::kStages;
         ok = bwd_wait(bars.empty(s), ((it / C::kStages) & 1u) ^ 1u, abort_flag, p);
@@ -305,7 +327,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     const uint32_t first = it > (uint32_t)C::kStages ? it - C::kStages : 0u;
     for (uint32_t r = first; r < it; ++r)
       bwd_wait(bars.full(r % C::kStages), (r / C::kStages) & 1u, abort_flag, p, false);
-    if (nu > 0) bwd_wait(bars.ab_full(), (nu - 1) & 1u, abort_flag, p, false);
+    if (!kDQ && nu > 0) bwd_wait(bars.ab_full(), (nu - 1) & 1u, abort_flag, p, false);
   } else if (warp == kBwdMmaWarp) {
     // ------------------------------------------------------- MMA issuer ---
     uint32_t it = 0, nu = 0, pw0 = 0, pw1 = 0;
@@ -314,8 +336,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     auto issue_sd = [&](int h, uint32_t n) {
       const uint32_t xb = sRing + (n % C::kStages) * 2 * C::kTileBytes;
       ptx::tc_fence_after();
-      bwd_mma_half<D>(tmem + C::s_col(h), sA, xb + 8192u * h);
-      bwd_mma_half<D>(tmem + C::g_col(h), sB, xb + C::kTileBytes + 8192u * h);
+      if constexpr (kDQ) {
+        bwd_mma_half_ts<D>(tmem + C::s_col(h), tmem + C::kTq, xb + 8192u * h);
+        bwd_mma_half_ts<D>(tmem + C::g_col(h), tmem + C::kTdo, xb + C::kTileBytes + 8192u * h);
+      } else {
+        bwd_mma_half<D>(tmem + C::s_col(h), sA, xb + 8192u * h);
+        bwd_mma_half<D>(tmem + C::g_col(h), sB, xb + C::kTileBytes + 8192u * h);
+      }
       if (ptx::elect_one()) ptx::mma_commit(bars.s_full(h));
       __syncwarp();
     };
@@ -408,6 +435,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       const int row = u.t * kBM + r;  // query row (kDQ) or key row
       float nlse2 = -INFINITY, delta = 0.f;
       if constexpr (kDQ) {
+        // This warpgroup's A operand row into tensor memory: Q (half 0) or
+        // dO (half 1), zeros past Nq, once the previous unit's MMAs are done.
+        ok = bwd_wait(bars.ab_empty(), (nu & 1u) ^ 1u, abort_flag, p);
+        if (!ok) break;
+        {
+          const __nv_bfloat16* src = h == 0 ? p.q : p.dout;
+          const uint4* arow = reinterpret_cast<const uint4*>(src + ((size_t)u.bh * p.Nq + (row < p.Nq ? row : 0)) * D);
+          const uint32_t tA = tmem + lane_base + (h == 0 ? C::kTq : C::kTdo);
+#pragma unroll
+          for (int ch = 0; ch < D / 64; ++ch) {
+            uint32_t a[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint4 x = row < p.Nq ? arow[8 * ch + i] : make_uint4(0u, 0u, 0u, 0u);
+              a[4 * i] = x.x;
+              a[4 * i + 1] = x.y;
+              a[4 * i + 2] = x.z;
+              a[4 * i + 3] = x.w;
+            }
+            ptx::tmem_st32(tA + 32 * ch, a);
+          }
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(bars.ab_full());
+        }
         // Per-row values: -log2(e) lse_i (or -inf for a row without keys),
         // D_i = dO_i . O_i, written once for the dK/dV launch.
         if (row < p.Nq) {
