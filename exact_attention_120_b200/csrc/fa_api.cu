@@ -254,6 +254,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((rc = encode_qkv_map(&p.tm_k, k, (int)bh, Nk, d, eb)) != FA_OK) return rc;
   if ((rc = encode_qkv_map(&p.tm_v, v, (int)bh, Nk, d, eb)) != FA_OK) return rc;
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_v8 = aligned(o, 32) ? 1 : 0;
   p.lse = lse;
   p.mask = block_mask;
   p.Nq = Nq;
@@ -506,6 +507,7 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   if ((rc = encode_varlen_map(&p.tm_k, k, total_k, H, d)) != FA_OK) return rc;
   if ((rc = encode_varlen_map(&p.tm_v, v, total_k, H, d)) != FA_OK) return rc;
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_v8 = aligned(o, 32) ? 1 : 0;
   p.lse = lse;
   p.mask = nullptr;
   p.Nq = max_seqlen_q;

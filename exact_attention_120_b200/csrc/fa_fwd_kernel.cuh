@@ -65,6 +65,7 @@ struct KernelParams {
   CUtensorMap tm_k;
   CUtensorMap tm_v;
   __nv_bfloat16* o;
+  int o_v8;  // o is 32-byte aligned: the epilogue may use 32-byte stores
   float* lse;
   const uint8_t* mask;  // nullptr or [B*H][nqt][nkt]
   int Nq;          // query rows per head
@@ -875,24 +876,35 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
       const size_t orow_i = kVarlen ? (size_t)(se.q0() + r) * p.heads + se.h() : (size_t)bh * p.Nq + r;
       const size_t lse_i = kVarlen ? (size_t)se.h() * p.total_q + se.q0() + r : (size_t)bh * p.Nq + r;
       uint4* orow = reinterpret_cast<uint4*>(p.o + orow_i * D);
+      // The whole O row in one tensor-memory round trip (the scores are dead
+      // here, so the registers are free), then 32-byte stores when O is
+      // 32-byte aligned.
+      uint32_t t[D / 32][32];
+      if (n > 0) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(tO + 32 * c, t[c]);
+        ptx::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) t[c][e] = 0u;
+      }
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t t[32];
-        if (n > 0) {
-          ptx::tmem_ld32(tO + 32 * c, t);
-          ptx::tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) t[e] = 0u;
-        }
         uint32_t pkd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          pkd[e] = ptx::pack_bf16x2(__uint_as_float(t[2 * e]) * inv, __uint_as_float(t[2 * e + 1]) * inv);
+          pkd[e] = ptx::pack_bf16x2(__uint_as_float(t[c][2 * e]) * inv, __uint_as_float(t[c][2 * e + 1]) * inv);
         if (in_range) {
+          if (p.o_v8) {
+            ptx::st_global_v8(orow + c * 4, pkd);
+            ptx::st_global_v8(orow + c * 4 + 2, pkd + 8);
+          } else {
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            orow[c * 4 + v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+            for (int v4 = 0; v4 < 4; ++v4)
+              orow[c * 4 + v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+          }
         }
       }
       if (in_range)
