@@ -83,3 +83,69 @@ def test_every_public_name_exists():
 
     missing = [n for n in fa.__all__ if not hasattr(fa, n)]
     assert not missing, missing
+
+
+def test_backward_argument_errors_before_any_cuda_call(lib):
+    p = 1 << 20  # never dereferenced: every case fails validation first
+    names = ["q", "k", "v", "o", "lse", "dout", "dq", "dk", "dv", "B", "H", "Nq", "Nk", "d", "scale",
+             "causal", "mask", "ws", "ws_bytes", "stream"]
+    base = [p, p * 2, p * 3, p * 4, p * 5, p * 6, p * 7, p * 8, p * 9, 1, 2, 300, 200, 64, 0.125, 0,
+            None, p * 10, 4096, None]
+
+    def call(**kw):
+        a = list(base)
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return fa.fa_bwd(*a)
+
+    for name in ("q", "k", "v", "o", "lse", "dout", "dq", "dk", "dv", "ws"):
+        assert call(**{name: None}) == fa.FA_ERR_INVALID_ARGUMENT, name
+    assert call(B=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(Nk=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(scale=float("nan")) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(causal=2) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(d=80) == fa.FA_ERR_UNSUPPORTED
+    assert call(dk=p * 8 + 4) == fa.FA_ERR_INVALID_ARGUMENT   # not 16-byte aligned
+    assert call(ws_bytes=100) == fa.FA_ERR_INVALID_ARGUMENT   # below 2*300*4 bytes of D
+    assert call(dq=p) == fa.FA_ERR_INVALID_ARGUMENT           # dq aliases q
+    assert call(dv=p * 8) == fa.FA_ERR_INVALID_ARGUMENT       # dv aliases dk
+    assert fa.fa_bwd_workspace_bytes(2, 3, 300) == 2 * 3 * 300 * 4
+    assert fa.fa_bwd_workspace_bytes(1, 1, 5) == 32          # rounded up to 16 bytes
+    assert fa.fa_bwd_workspace_bytes(0, 1, 5) == 0
+
+
+def test_varlen_and_fp8_argument_errors_before_any_cuda_call(lib):
+    p = 1 << 20
+    # fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_seqlen_q, d, scale, causal, stream)
+    vbase = [p, p * 2, p * 3, p * 4, p * 5, p * 6, p * 7, 2, 4, 100, 100, 60, 128, 0.1, 1, None]
+    vnames = ["q", "k", "v", "o", "lse", "cu_q", "cu_k", "B", "H", "tq", "tk", "maxq", "d", "scale",
+              "causal", "stream"]
+
+    def vcall(**kw):
+        a = list(vbase)
+        for key, val in kw.items():
+            a[vnames.index(key)] = val
+        return fa.fa_fwd_varlen(*a)
+
+    assert vcall(cu_q=None) == fa.FA_ERR_INVALID_ARGUMENT
+    assert vcall(tq=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert vcall(maxq=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert vcall(cu_k=p * 7 + 2) == fa.FA_ERR_INVALID_ARGUMENT  # offsets not 4-byte aligned
+    assert vcall(o=p * 2) == fa.FA_ERR_INVALID_ARGUMENT         # o aliases k
+    assert vcall(d=32) == fa.FA_ERR_UNSUPPORTED
+    # fa_fwd_fp8(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, mask, qd, kd, vd, stream)
+    fbase = [p, p * 2, p * 3, p * 4, p * 5, 1, 1, 128, 128, 128, 0.1, 0, None, 1.0, 1.0, 1.0, None]
+    fnames = ["q", "k", "v", "o", "lse", "B", "H", "Nq", "Nk", "d", "scale", "causal", "mask", "qd",
+              "kd", "vd", "stream"]
+
+    def fcall(**kw):
+        a = list(fbase)
+        for key, val in kw.items():
+            a[fnames.index(key)] = val
+        return fa.fa_fwd_fp8(*a)
+
+    assert fcall(qd=0.0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert fcall(kd=float("inf")) == fa.FA_ERR_INVALID_ARGUMENT
+    assert fcall(vd=-1.0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert fcall(d=64) == fa.FA_ERR_UNSUPPORTED                 # 8-bit inputs need d = 128
+    assert fcall(v=None) == fa.FA_ERR_INVALID_ARGUMENT
