@@ -15,8 +15,13 @@
 // block, streaming all of K and V), with two Q blocks sharing each K/V tile.
 // The grid is persistent: CTA c takes work units c, c + gridDim.x, ...
 //
+// Instantiations: Cfg<D, fp8> for head dim 64 or 128 with bf16 inputs, or
+// d = 128 with e4m3 inputs (tcgen05 kind::f8f6f4); kVarlen for packed
+// variable-length batches.  One source, the same roles and barriers.
+//
 // Warp roles (384 threads, one CTA per SM, 512 tensor-memory columns):
-//   warp  0    MMA issue (one thread): S_q = Q_q K_j^T and O_q += P_q V_j
+//   warp  0    MMA issue (warp-uniform loop, one elected lane issues):
+//              S_q = Q_q K_j^T and O_q += P_q V_j
 //   warp  1    TMA producer: Q tiles, then K_j, V_j through a ring in smem
 //   warps 2-3  idle
 //   warps 4-7  softmax for query tile 2p   (thread t owns row t of the tile)
@@ -26,16 +31,18 @@
 //
 // Tensor memory (fp32 columns, lane = tile row):
 //   S_0 [0,128)  S_1 [128,256)  O_0 [256,256+D)  O_1 [384,384+D)
-//   P_q (bf16 pairs, 64 columns) overwrites the first half of S_q once the
-//   softmax has read S_q into registers; the PV MMA reads P_q from there.
+//   d = 128: P_q (bf16 pairs in 64 columns, or e4m3 quads in 32) overwrites
+//   the start of S_q once the softmax has read S_q into registers; the PV
+//   MMA reads P_q from there.  d = 64: O_q takes 64 columns and P_q gets its
+//   own ([384,448), [448,512)), so the next S_q can run during the softmax.
 //
 // Online softmax in base 2: with c = scale * log2(e), each row keeps a
 // reference max m_ref (in units of c * score) and l = sum 2^(c s - m_ref).
 // The reference is moved (and O, l rescaled by 2^(m_old - m_new), the
 // concatenation rule of "理解 Flash Attention", "瓦片注意力计算") only when the
-// tile max exceeds it by more than kRescaleLog2 -- otherwise p <= 2^8, which
-// fp32 and bf16 hold without loss.  l sums the bf16-rounded p that the PV MMA
-// consumes, so O / l is an exact convex combination of V rows.
+// tile max exceeds it by more than Cfg::kRescale (2^8 for bf16 P, so p <= 2^8;
+// e4m3 P moves at 2^4 with a 2^4 shift, see Cfg).  l sums the rounded p that
+// the PV MMA consumes, so O / l is an exact convex combination of V rows.
 //
 // Every wait on an mbarrier is bounded (globaltimer); on expiry the CTA
 // records FA_ERR_DEVICE_TIMEOUT, all roles leave their loops, in-flight TMA
@@ -56,7 +63,6 @@ constexpr int kThreads = 384;
 constexpr int kMmaWarp = 0;
 constexpr int kLoadWarp = 1;
 constexpr int kFirstSoftmaxWarp = 4;
-constexpr float kRescaleLog2 = 8.0f;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStatusTimeout = 4;  // == FA_ERR_DEVICE_TIMEOUT
 
@@ -217,7 +223,7 @@ struct Cfg {
 // polynomial fitted for minimum relative error (max 7.6e-5, well under the
 // bf16 rounding that follows; the fit is exact_attention_120_b200/exp2_poly_fit.py);
 // 2^n added to the exponent field.  Arguments below -125 (masked scores are
-// -inf) give 2^-125.  Arguments never exceed +8 here (see kRescaleLog2).
+// -inf) give 2^-125.  Arguments never exceed +8 here (see Cfg::kRescale).
 constexpr float kExp2Clamp = -125.0f;
 constexpr float kExp2Round = 12582912.0f;  // 1.5 * 2^23
 constexpr float kExp2C0 = 9.999282360e-01f;
@@ -749,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
           const float tmax = ptx::max3(fmaxf(mx[0], mx[1]), mx[2], mx[3]);
           const float m_new = fmaxf(m_ref, tmax * sl);
           // Move the reference max only when the new one exceeds it by more than
-          // 2^kRescaleLog2 (always on the first visible tile: m_ref = -inf).
+          // 2^kRescale (always on the first visible tile: m_ref = -inf).
           const bool rescale = m_new > m_ref + C::kRescale;
           float alpha = 1.f;
           if (rescale) {
