@@ -1,9 +1,10 @@
 // Host side of the C ABI declared in include/fa.h: argument validation,
 // TMA descriptor encoding, per-device set-up and the kernel launch.
 //
-// Nothing here computes any part of attention; every step of the forward
-// pass runs in fa_fwd_kernel.  There is no CPU fallback: without an sm_100
-// device the entry points return FA_ERR_UNSUPPORTED.
+// Nothing here computes any part of attention: every step runs in the
+// kernels (fa_fwd_kernel and its instantiations, fa_combine_kernel for split
+// keys, fa_bwd_kernel for the gradients).  There is no CPU fallback: without
+// an sm_100 device the entry points return FA_ERR_UNSUPPORTED.
 
 #include <cuda.h>
 #include <cuda_runtime.h>

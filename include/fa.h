@@ -1,5 +1,9 @@
 /*
- * fa.h -- C ABI of the B200 (sm_100a) fused exact-attention forward pass.
+ * fa.h -- C ABI of the B200 (sm_100a) fused exact-attention kernels: the
+ * forward pass (fa_fwd and its variants for different query/key lengths,
+ * split keys, variable-length batches and 8-bit inputs) and the backward
+ * pass (fa_bwd).  The common definitions follow; each variant states what it
+ * adds or changes at its declaration.
  *
  * The operation
  * -------------
