@@ -266,7 +266,10 @@ FA_API const char* fa_status_string(int status);
 /* The cudaError_t value behind the last FA_ERR_CUDA on this host thread. */
 FA_API int fa_last_cuda_error(void);
 
-/* Number of kernel launches one fa_fwd / fa_fwd_qk call makes (constant: 1). */
+/* Number of kernel launches one fa_fwd / fa_fwd_qk / fa_fwd_varlen /
+ * fa_fwd_fp8 call makes (constant: 1).  fa_fwd_splitkv with more than one
+ * slice makes 2 (the forward and the merge), fa_bwd makes 2 (the dQ and the
+ * dK/dV launches). */
 FA_API int fa_launches_per_call(void);
 
 #ifdef __cplusplus
