@@ -37,6 +37,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -77,10 +78,16 @@ def load_peaks():
 
 
 def kernel_hash(sources=KERNEL_SOURCES) -> str:
+    """Hash of the kernel sources' code: comments and whitespace are dropped,
+    so a comment edit keeps the recorded counters while any code change
+    invalidates them."""
     h = hashlib.sha256()
     for rel in sources:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
