@@ -607,6 +607,18 @@ def run_ours(args, info):
     if st != fa.FA_OK:
         raise fa.FaError(st, "device status after timed region")
 
+    # ---- per-step distribution (outside the timed region): one event pair per step
+    per = []
+    for _ in range(min(args.steps, 50)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        job.launch()
+        b.record(stream)
+        per.append((a, b))
+    torch.cuda.synchronize(dev)
+    per_ms = sorted(a.elapsed_time(b) for a, b in per)
+    pct = lambda f: per_ms[min(len(per_ms) - 1, int(f * len(per_ms)))]  # noqa: E731
+
     # ---- end to end: pinned host inputs -> device -> public API -> host outputs
     h2d, d2h = job.host_buffers()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -660,6 +672,8 @@ def run_ours(args, info):
                      "flops_per_launch": flops},
         "e2e": {"value": info.world_size * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "ms_per_step_percentiles": {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9),
+                                    "steps": len(per_ms)},
         "gpu_launches": args.steps * job.launches_per_step,
         "clocks": clocks,
         "cpu_baseline": cpu,
