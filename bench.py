@@ -343,6 +343,7 @@ class BwdJob(FwdJob):
     name = "bwd"
     metric = "fused attention bwd TFLOP/s (bf16 dQ, dK, dV; 2.5x forward FLOPs) and % of dense BF16 peak"
     kernel_sources = ("exact_attention_120_b200/csrc/fa_bwd_kernel.cuh",
+                      "exact_attention_120_b200/csrc/fa_fwd_kernel.cuh",  # shared helpers
                       "exact_attention_120_b200/csrc/ptx.cuh",
                       "exact_attention_120_b200/csrc/fa_api.cu")
 

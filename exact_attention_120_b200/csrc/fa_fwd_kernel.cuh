@@ -214,6 +214,12 @@ struct Cfg {
   // reference survive the rounding.
   static constexpr float kRescale = kFp8_ ? 4.0f : 8.0f;
   static constexpr float kPShift = kFp8_ ? 4.0f : 0.0f;
+  // One pair in kPolyEvery of each row's exp2 goes through exp2_poly2 on the
+  // FMA pipe, the rest through MUFU.  Measured on B200 (A/B on one GPU):
+  // bf16 runs best at 1 in 8 (+0.6 to +2.2 % over 1 in 4; 1 in 3 or more, or
+  // none at all, is slower); e4m3, whose MMAs take half the time and leave
+  // the softmax more MUFU-bound, at 1 in 4 (1 in 8 is 3 % slower there).
+  static constexpr int kPolyEvery = kFp8_ ? 4 : 8;
 };
 
 // 2^x on the FMA pipe for two lanes (relieves the MUFU exp2 unit, which at
@@ -224,6 +230,7 @@ struct Cfg {
 // bf16 rounding that follows; the fit is exact_attention_120_b200/exp2_poly_fit.py);
 // 2^n added to the exponent field.  Arguments below -125 (masked scores are
 // -inf) give 2^-125.  Arguments never exceed +8 here (see Cfg::kRescale).
+// Cfg::kPolyEvery sets how many pairs take this path.
 constexpr float kExp2Clamp = -125.0f;
 constexpr float kExp2Round = 12582912.0f;  // 1.5 * 2^23
 constexpr float kExp2C0 = 9.999282360e-01f;
@@ -245,8 +252,6 @@ __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float
   y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
-// One pair in kPolyEvery of each row's exp2 goes through exp2_poly2.
-constexpr int kPolyEvery = 4;
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, A K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
@@ -786,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
               const int cc = 32 * half + c;
               float x0, x1, p0, p1;
               ptx::fma2(x0, x1, s[2 * cc], s[2 * cc + 1], sl, sl, neg_m, neg_m);
-              if (cc % kPolyEvery == kPolyEvery - 1) {
+              if (cc % C::kPolyEvery == C::kPolyEvery - 1) {
                 exp2_poly2(p0, p1, x0, x1);
               } else {
                 p0 = ptx::ex2(x0);
