@@ -1,9 +1,12 @@
-"""B200 (sm_100a) fused exact-attention forward: Python binding of the C ABI.
+"""B200 (sm_100a) fused exact attention: Python binding of the C ABI.
 
-The binding only marshals arguments: every step of the forward pass runs in
-the CUDA kernel behind ``libfa_b200.so`` (see ``include/fa.h``).  PyTorch is
-used for device memory and streams.  There is no CPU fallback: if the
-library is missing or the device is not an sm_100 GPU the calls raise.
+The binding only marshals arguments: every step of the forward and backward
+passes runs in the CUDA kernels behind ``libfa_b200.so`` (see
+``include/fa.h``).  PyTorch is used for device memory and streams.  There is
+no CPU fallback: if the library is missing or the device is not an sm_100
+GPU the calls raise.  The tensor-level functions check every tensor's dtype,
+device, contiguity and shape before anything is launched (the C ABI takes raw
+pointers and cannot).
 
 Functions with the C names take raw device addresses:
 
@@ -14,10 +17,13 @@ Functions with the C names take raw device addresses:
   ``fa_fwd_splitkv_workspace_bytes`` and ``fa_fwd_splitkv_heuristic``
 * ``fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, causal,
   block_mask, workspace, workspace_bytes, stream)`` and ``fa_bwd_workspace_bytes``
+* ``fa_fwd_varlen(...)``, ``fa_fwd_fp8(...)``
 * ``fa_device_status(stream)``, ``fa_status_string(status)``
 
-and ``attention_forward(q, k, v, ...)`` is the tensor-level convenience that
-allocates ``o`` and ``lse`` and launches on torch's current stream.
+Tensor-level functions (allocate outputs with torch, launch on torch's current
+stream): ``attention_forward``, ``attention_forward_splitkv``,
+``attention_forward_varlen``, ``attention_forward_fp8`` and
+``attention_backward``.
 """
 
 from __future__ import annotations
@@ -160,6 +166,42 @@ def fa_launches_per_call() -> int:
     return load_library().fa_launches_per_call()
 
 
+def _check(t, name, dtype, shape, device=None):
+    """Raise ValueError unless `t` is a contiguous CUDA tensor of `dtype` and
+    `shape` (on `device` when given)."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+
+
+def _check_qkv(q, k, v, dtype):
+    """q [B, H, Nq, d], k and v [B, H, Nk, d] of `dtype` on one device."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q must be [B, H, Nq, d] and k, v [B, H, Nk, d]")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    _check(q, "q", dtype, (B, H, Nq, d))
+    _check(k, "k", dtype, (B, H, Nk, d), q.device)
+    _check(v, "v", dtype, (B, H, Nk, d), q.device)
+    return B, H, Nq, Nk, d
+
+
+def _check_mask(block_mask, B, H, Nq, Nk, device):
+    if block_mask is None:
+        return None
+    nbq = (Nq + MASK_BLOCK - 1) // MASK_BLOCK
+    nbk = (Nk + MASK_BLOCK - 1) // MASK_BLOCK
+    import torch
+
+    _check(block_mask, "block_mask", torch.uint8, (B, H, nbq, nbk), device)
+    return block_mask.data_ptr()
+
+
 def attention_forward(q, k, v, causal=False, block_mask=None, scale=None, out=None, lse=None,
                       stream=None):
     """O, lse = attention(q, k, v) through the C ABI.
@@ -172,28 +214,16 @@ def attention_forward(q, k, v, causal=False, block_mask=None, scale=None, out=No
     """
     import torch
 
-    if q.dim() != 4 or k.shape != v.shape or k.dim() != 4 or q.shape[:2] != k.shape[:2] \
-            or q.shape[3] != k.shape[3]:
-        raise ValueError("q must be [B, H, Nq, d] and k, v [B, H, Nk, d]")
-    for t in (q, k, v):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v must be contiguous CUDA bfloat16 tensors")
-    B, H, Nq, d = q.shape
-    Nk = k.shape[2]
+    B, H, Nq, Nk, d = _check_qkv(q, k, v, torch.bfloat16)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    mask_ptr = None
-    if block_mask is not None:
-        nbq = (Nq + MASK_BLOCK - 1) // MASK_BLOCK
-        nbk = (Nk + MASK_BLOCK - 1) // MASK_BLOCK
-        if (block_mask.dtype != torch.uint8 or not block_mask.is_cuda
-                or tuple(block_mask.shape) != (B, H, nbq, nbk) or not block_mask.is_contiguous()):
-            raise ValueError(f"block_mask must be a contiguous CUDA uint8 [B,H,{nbq},{nbk}] tensor")
-        mask_ptr = block_mask.data_ptr()
+    _check(out, "out", torch.bfloat16, (B, H, Nq, d), q.device)
+    _check(lse, "lse", torch.float32, (B, H, Nq), q.device)
+    mask_ptr = _check_mask(block_mask, B, H, Nq, Nk, q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     with torch.cuda.device(q.device):
@@ -219,20 +249,24 @@ def attention_forward_splitkv(q, k, v, causal=False, block_mask=None, scale=None
     """
     import torch
 
-    B, H, Nq, d = q.shape
-    Nk = k.shape[2]
+    B, H, Nq, Nk, d = _check_qkv(q, k, v, torch.bfloat16)
     if num_splits is None:
         num_splits = fa_fwd_splitkv_heuristic(B, H, Nq, Nk)
     need = fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None and (not workspace.is_cuda or not workspace.is_contiguous()
+                                  or workspace.device != q.device):
+        raise ValueError("workspace must be a contiguous CUDA tensor on q's device")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    mask_ptr = None if block_mask is None else block_mask.data_ptr()
+    _check(out, "out", torch.bfloat16, (B, H, Nq, d), q.device)
+    _check(lse, "lse", torch.float32, (B, H, Nq), q.device)
+    mask_ptr = _check_mask(block_mask, B, H, Nq, Nk, q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     ws_ptr = None if workspace is None else workspace.data_ptr()
@@ -277,18 +311,19 @@ def attention_backward(q, k, v, o, lse, dout, causal=False, block_mask=None, sca
     """
     import torch
 
-    B, H, Nq, d = q.shape
-    Nk = k.shape[2]
+    B, H, Nq, Nk, d = _check_qkv(q, k, v, torch.bfloat16)
+    _check(o, "o", torch.bfloat16, (B, H, Nq, d), q.device)
+    _check(dout, "dout", torch.bfloat16, (B, H, Nq, d), q.device)
+    _check(lse, "lse", torch.float32, (B, H, Nq), q.device)
+    mask_ptr = _check_mask(block_mask, B, H, Nq, Nk, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    for t in (q, k, v, o, dout):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v, o, dout must be contiguous CUDA bfloat16 tensors")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     need = fa_bwd_workspace_bytes(B, H, Nq)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    mask_ptr = None if block_mask is None else block_mask.data_ptr()
+    if not workspace.is_cuda or not workspace.is_contiguous() or workspace.device != q.device:
+        raise ValueError("workspace must be a contiguous CUDA tensor on q's device")
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     with torch.cuda.device(q.device):
@@ -313,23 +348,26 @@ def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
     """
     import torch
 
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q must be [total_q, H, d] and k, v [total_k, H, d]")
     Tq, H, d = q.shape
     Tk = k.shape[0]
+    _check(q, "q", torch.bfloat16, (Tq, H, d))
+    _check(k, "k", torch.bfloat16, (Tk, H, d), q.device)
+    _check(v, "v", torch.bfloat16, (Tk, H, d), q.device)
+    if cu_seqlens_q.dim() != 1 or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q must hold B + 1 >= 2 offsets")
+    B = cu_seqlens_q.numel() - 1
+    _check(cu_seqlens_q, "cu_seqlens_q", torch.int32, (B + 1,), q.device)
+    _check(cu_seqlens_k, "cu_seqlens_k", torch.int32, (B + 1,), q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    for t in (q, k, v):
-        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v must be contiguous CUDA bfloat16 tensors")
-    for t in (cu_seqlens_q, cu_seqlens_k):
-        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("cu_seqlens must be contiguous CUDA int32 tensors")
-    B = cu_seqlens_q.numel() - 1
-    if cu_seqlens_k.numel() != B + 1:
-        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((H, Tq), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.bfloat16, (Tq, H, d), q.device)
+    _check(lse, "lse", torch.float32, (H, Tq), q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     with torch.cuda.device(q.device):
@@ -351,18 +389,24 @@ def attention_forward_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal=Fa
     """
     import torch
 
+    if q8.dim() != 4 or k8.dim() != 4:
+        raise ValueError("q8 must be [B, H, Nq, d] and k8, v8 [B, H, Nk, d]")
+    codes = (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8))
     B, H, Nq, d = q8.shape
     Nk = k8.shape[2]
+    for t, name, shape in ((q8, "q8", (B, H, Nq, d)), (k8, "k8", (B, H, Nk, d)), (v8, "v8", (B, H, Nk, d))):
+        if t.dtype not in codes:
+            raise ValueError(f"{name} must hold E4M3 codes (uint8 or float8_e4m3fn)")
+        _check(t, name, t.dtype, shape, q8.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    for t in (q8, k8, v8):
-        if t.element_size() != 1 or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q8, k8, v8 must be contiguous CUDA 8-bit tensors")
     if out is None:
         out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q8.device)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q8.device)
-    mask_ptr = None if block_mask is None else block_mask.data_ptr()
+    _check(out, "out", torch.bfloat16, (B, H, Nq, d), q8.device)
+    _check(lse, "lse", torch.float32, (B, H, Nq), q8.device)
+    mask_ptr = _check_mask(block_mask, B, H, Nq, Nk, q8.device)
     if stream is None:
         stream = torch.cuda.current_stream(q8.device).cuda_stream
     with torch.cuda.device(q8.device):
