@@ -1,7 +1,7 @@
 """The bench.py contract, checked without a GPU.
 
 * The reference arm (the float64 oracle on host cores) prints one JSON line
-  with the keys the driver reads, a cpu_baseline and an e2e object.
+  with the contract keys, a cpu_baseline and an e2e object.
 * The GPU arm refuses to run without CUDA instead of falling back to a CPU
   path.
 * Argument checks: at least 3 warm-up steps; the reference arm is forward only.
