@@ -8,10 +8,11 @@
 //   dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Two launches of one kernel template, no atomics:
-//  * kDQ = true, stationary on a 128-row query tile (Q, dO in shared memory):
-//    per visible key tile j, S = Q K_j^T and dP = dO V_j^T, then the
-//    elementwise dS (one thread per query row, bf16 written over S), then
-//    dQ += dS K_j.  It also writes D_i to the workspace for the second launch.
+//  * kDQ = true, stationary on a 128-row query tile (Q, dO copied into tensor
+//    memory by the elementwise warpgroups, as the A operands): per visible
+//    key tile j, S = Q K_j^T and dP = dO V_j^T, then the elementwise dS (one
+//    thread per query row, bf16 written over S), then dQ += dS K_j.  It also
+//    writes D_i to the workspace for the second launch.
 //  * kDQ = false, stationary on a 128-key tile (K, V): per query tile i that
 //    sees it, S^T = K Q_i^T and dP^T = V dO_i^T, the elementwise P^T and dS^T
 //    (one thread per key row), then dV += P^T dO_i and dK += dS^T Q_i.
