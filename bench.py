@@ -172,10 +172,12 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def oracle_sample(w, q, k, v, mask, rows_per_chunk, budget_s=None, max_chunks=None, start=0):
+def oracle_sample(w, q, k, v, mask, rows_per_chunk, budget_s=None, max_chunks=None, start=0,
+                  keep=None):
     """Time the float64 oracle on successive chunks of query rows of the
     workload (head-major order), until `budget_s` seconds or `max_chunks`.
-    Returns (useful_flops, seconds, rows)."""
+    Returns (useful_flops, seconds, rows).  With a list `keep`, appends each
+    chunk's (sample, o, lse) to it."""
     import numpy as np
 
     import oracle
@@ -190,9 +192,11 @@ def oracle_sample(w, q, k, v, mask, rows_per_chunk, budget_s=None, max_chunks=No
         idx = [(r0 + i) % total_rows for i in range(rows_per_chunk)]
         sample = [(i // (w.H * w.N), (i // w.N) % w.H, i % w.N) for i in idx]
         t0 = time.perf_counter()
-        oracle.attention_ref_rows(q, k, v, w.scale, sample, causal=w.causal,
-                                  block_mask=None if mask is None else mask)
+        ref = oracle.attention_ref_rows(q, k, v, w.scale, sample, causal=w.causal,
+                                        block_mask=None if mask is None else mask)
         t_total += time.perf_counter() - t0
+        if keep is not None:
+            keep.append((sample, ref[0], ref[1]))
         for (b, h, i) in sample:
             vis = oracle.visible_mask(w.N, w.N, w.causal,
                                       None if mask is None else mask[b, h], rows=np.array([i]))
@@ -329,10 +333,33 @@ class FwdJob:
     def cpu_baseline(self, args):
         w = self.w
         qn, kn, vn, mn = numpy_inputs(self.q, self.k, self.v, self.mask)
-        f, t, rows = oracle_sample(w, qn, kn, vn, mn, args.cpu_rows, budget_s=args.cpu_budget)
+        kept = []
+        f, t, rows = oracle_sample(w, qn, kn, vn, mn, args.cpu_rows, budget_s=args.cpu_budget,
+                                   keep=kept)
+        self.parity = self._parity(kept)
         return {"value": f / t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                 "sample": f"{rows} query rows of {w.name} (complete rows over all N={w.N} keys, "
                           f"head-major from row 0), {t:.1f} s of float64 NumPy/BLAS oracle"}
+
+    def _parity(self, kept):
+        """max |O - O_ref| and |lse - lse_ref| of the timed run's output on the
+        rows the oracle computed (after the timed region, untimed)."""
+        import numpy as np
+        import torch
+
+        o = self.od.to("cpu", torch.float64).numpy()
+        lse = self.ld.to("cpu", torch.float64).numpy()
+        e_o = e_l = 0.0
+        n = 0
+        for sample, o_ref, l_ref in kept:
+            b, h, i = (np.array(x) for x in zip(*sample))
+            e_o = max(e_o, float(np.max(np.abs(o[b, h, i] - o_ref))))
+            fin = np.isfinite(l_ref)
+            if fin.any():
+                e_l = max(e_l, float(np.max(np.abs(lse[b, h, i][fin] - l_ref[fin]))))
+            n += len(sample)
+        return {"rows": n, "max_abs_dO": e_o, "max_abs_dlse": e_l, "bar": {"dO": 2e-2, "dlse": 1e-2},
+                "within_bar": e_o <= 2e-2 and e_l <= 1e-2}
 
 
 class BwdJob(FwdJob):
@@ -679,7 +706,11 @@ def run_ours(args, info):
         "clocks": clocks,
         "cpu_baseline": cpu,
         "kernel_hash": khash,
+        "device": {"name": torch.cuda.get_device_name(dev), "torch": torch.__version__,
+                   "cuda": torch.version.cuda},
     }
+    if getattr(job, "parity", None) is not None:
+        line["parity_sample"] = job.parity
     if job.name == "bwd":
         line["config"]["pass"] = "backward (fa_bwd: dQ kernel then dK/dV kernel)"
     print(json.dumps(line), flush=True)
