@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
-SOURCES = [os.path.join(CSRC, "fa_api.cu")]
+SOURCES = [os.path.join(CSRC, "fa_api.cu"), os.path.join(CSRC, "fa_layout_checks.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("fa_fwd_kernel.cuh", "fa_combine.cuh", "fa_bwd_kernel.cuh", "ptx.cuh")] + [
     os.path.join(INCLUDE, "fa.h"), os.path.join(INCLUDE, "fa_testing.h")]
 
