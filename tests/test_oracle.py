@@ -421,6 +421,9 @@ def test_qk_lengths_brute_force(nq, nk, mode):
     np.testing.assert_allclose(l2, lse, rtol=1e-12, atol=1e-13)
 
 
+# With nq > nk the library warns that fully masked rows come out NaN; those
+# rows are excluded from the comparison below.
+@pytest.mark.filterwarnings("ignore:Lower right causal bias will produce NaNs")
 @pytest.mark.parametrize("nq,nk", [(5, 40), (40, 40), (33, 17)])
 def test_qk_causal_matches_lower_right_sdpa(nq, nk):
     """PyTorch's lower-right causal bias is the same bottom-right alignment."""
