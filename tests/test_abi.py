@@ -149,3 +149,43 @@ def test_varlen_and_fp8_argument_errors_before_any_cuda_call(lib):
     assert fcall(vd=-1.0) == fa.FA_ERR_INVALID_ARGUMENT
     assert fcall(d=64) == fa.FA_ERR_UNSUPPORTED                 # 8-bit inputs need d = 128
     assert fcall(v=None) == fa.FA_ERR_INVALID_ARGUMENT
+
+
+def _c_prototypes():
+    """Name -> (return type, [parameter types]) of every FA_API declaration."""
+    protos = {}
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for ret, name, params in re.findall(r"FA_API\s+([\w\s\*]+?)\s*\b(fa_\w+)\s*\(([^)]*)\)\s*;",
+                                            text):
+            params = " ".join(params.split())
+            types = [] if params in ("", "void") else \
+                [re.sub(r"\s*\b\w+$", "", p.strip()) for p in params.split(",")]
+            protos[name] = (" ".join(ret.split()), types)
+    return protos
+
+
+def _ctype_of(c_type):
+    c_type = c_type.replace("const ", "").strip()
+    if c_type.endswith("*"):
+        return ctypes.c_char_p if c_type == "char*" else ctypes.c_void_p
+    return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t,
+            "unsigned long long": ctypes.c_ulonglong}[c_type]
+
+
+def test_binding_signatures_match_the_headers():
+    """Every ctypes signature the binding installs has the C prototype's
+    parameter count and, position by position, the same kind of argument
+    (pointer, int, float, size_t, 64-bit integer) and return type."""
+    protos = _c_prototypes()
+    assert set(protos) == _declared_functions()
+    assert set(fa._SIGNATURES) == set(protos)
+    for name, (ret, params) in protos.items():
+        res, args = fa._SIGNATURES[name]
+        assert res is _ctype_of(ret), (name, ret)
+        assert len(args) == len(params), (name, len(args), len(params))
+        for i, (got, want) in enumerate(zip(args, params)):
+            assert got is _ctype_of(want), (name, i, want)
