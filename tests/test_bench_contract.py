@@ -4,6 +4,8 @@
   with the contract keys, a cpu_baseline and an e2e object.
 * The GPU arm refuses to run without CUDA instead of falling back to a CPU
   path.
+* Under a multi-rank launch the reference arm runs on rank 0 alone; the other
+  ranks exit 0 without work or output.
 * Argument checks: at least 3 warm-up steps; the reference arm is forward only.
 """
 
@@ -46,6 +48,20 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"].startswith("small")
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    args = ("--impl", "reference", "--gpus", "2", "--workload", "small", "--steps", "1",
+            "--warmup", "3", "--reference-rows", "32")
+    other = _run(*args, env={"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
+    assert other.returncode == 0, other.stderr
+    assert other.stdout.strip() == ""
+    root = _run(*args, env={"RANK": "0", "LOCAL_RANK": "0", "WORLD_SIZE": "2"})
+    assert root.returncode == 0, root.stderr
+    lines = [ln for ln in root.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU refusal")
