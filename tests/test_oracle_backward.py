@@ -113,3 +113,48 @@ def test_delta_is_row_dot():
     o = _r(1).normal(size=(1, 2, 5, 3))
     do = _r(2).normal(size=(1, 2, 5, 3))
     np.testing.assert_allclose(oracle.softmax_delta(o, do), np.einsum("bhnd,bhnd->bhn", o, do))
+
+
+# Plausible mistakes planted in a copy of the gradient oracle (on the CPU): a
+# dropped or sign-flipped row term, a missing scale, a swapped operand, the
+# mask left out.  Each must make at least one pin above fail.
+PLANTED = {
+    "drop_delta": ("ds = p * (dp - dd[:, None])", "ds = p * dp"),
+    "delta_sign": ("ds = p * (dp - dd[:, None])", "ds = p * (dp + dd[:, None])"),
+    "dq_no_scale": ("dq[b, h] = scale * (ds @ k[b, h])", "dq[b, h] = ds @ k[b, h]"),
+    "dq_uses_v": ("dq[b, h] = scale * (ds @ k[b, h])", "dq[b, h] = scale * (ds @ v[b, h])"),
+    "dv_uses_o": ("dv[b, h] = p.T @ do[b, h]", "dv[b, h] = p.T @ o"),
+    "delta_from_q": ("dd = np.sum(do[b, h] * o, axis=1)", "dd = np.sum(do[b, h] * q[b, h], axis=1)"),
+    "dk_uses_do": ("dk[b, h] = scale * (ds.T @ q[b, h])", "dk[b, h] = scale * (ds.T @ do[b, h])"),
+    "mask_ignored": ("s = np.where(vis, s, -np.inf)", "s = s"),
+}
+
+
+def _bwd_mutant(old, new):
+    import inspect
+
+    from oracle import backward as bwd_mod
+
+    src = inspect.getsource(bwd_mod.attention_bwd_ref)
+    assert src.count(old) == 1, old
+    ns = dict(vars(bwd_mod))
+    exec(compile(src.replace(old, new), bwd_mod.__file__, "exec"), ns)
+    return ns["attention_bwd_ref"]
+
+
+@pytest.mark.parametrize("kind", sorted(PLANTED))
+def test_planted_gradient_mistakes_are_caught(kind, monkeypatch):
+    monkeypatch.setattr(oracle, "attention_bwd_ref", _bwd_mutant(*PLANTED[kind]))
+    pins = [lambda: test_gradients_match_finite_differences("sparse_causal", 3, 6),
+            lambda: test_gradients_match_finite_differences("full", 5, 5),
+            lambda: test_gradients_match_torch_autograd(8, 20, True),
+            test_constant_values_give_no_query_key_gradient,
+            lambda: test_softmax_gradient_rows_sum_to_zero("causal"),
+            test_invisible_keys_get_no_gradient]
+    failed = 0
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed > 0, f"no pin caught the planted mistake {kind!r}"
