@@ -111,3 +111,46 @@ def test_rounding_bound_holds(seed):
         pt = p * (1 + e)
         o2 = (pt @ v[0, 0]) / pt.sum(axis=1, keepdims=True)
         assert np.all(np.abs(o2 - o[0, 0]) <= u / (1 - u) * sp[0, 0] + 1e-12)
+
+
+# Plausible mistakes planted in a copy of the 8-bit oracle (on the CPU); each
+# must make at least one pin above fail.
+PLANTED = {
+    "bias_8": ("np.exp2(e.astype(np.float64) - 7.0)", "np.exp2(e.astype(np.float64) - 8.0)"),
+    "subnormal_exp": ("(m / 8.0) * 2.0 ** -6", "(m / 8.0) * 2.0 ** -7"),
+    "subnormal_implicit_one": ("sub = sign * (m / 8.0)", "sub = sign * (1.0 + m / 8.0)"),
+    "mantissa_16ths": ("(1.0 + m / 8.0) * np.exp2", "(1.0 + m / 16.0) * np.exp2"),
+    "nan_as_max": ("np.where((c & 0x7F) == 0x7F, np.nan, out)", "out"),
+    "v_takes_k_scale": ("e4m3_decode(v8) * float(v_descale)", "e4m3_decode(v8) * float(k_descale)"),
+    "q_unscaled": ("e4m3_decode(q8) * float(q_descale)", "e4m3_decode(q8)"),
+}
+
+
+def _fp8_mutant(kind, monkeypatch):
+    import inspect
+
+    from oracle import fp8 as fp8_mod
+
+    old, new = PLANTED[kind]
+    for name in ("e4m3_decode", "attention_fp8_ref"):
+        src = inspect.getsource(getattr(fp8_mod, name))
+        if old in src:
+            ns = dict(vars(fp8_mod))
+            exec(compile(src.replace(old, new), fp8_mod.__file__, "exec"), ns)
+            monkeypatch.setattr(oracle, name, ns[name])
+            return
+    raise AssertionError(f"{old!r} not found")
+
+
+@pytest.mark.parametrize("kind", sorted(PLANTED))
+def test_planted_fp8_mistakes_are_caught(kind, monkeypatch):
+    _fp8_mutant(kind, monkeypatch)
+    pins = [test_e4m3_closed_forms, test_e4m3_all_codes_match_torch,
+            lambda: test_fp8_attention_matches_brute(True)]
+    failed = 0
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed > 0, f"no pin caught the planted mistake {kind!r}"
