@@ -5,8 +5,10 @@
   keys and more queries than keys, full and causal.
 * Sequences are independent: changing one sequence's tokens leaves every
   other sequence's outputs bit-identical.
-* A planted mistake (attending across sequence boundaries) fails the
-  brute-force pin.
+* Planted mistakes fail a pin: attending across sequence boundaries, and
+  mutants planted in a copy of the oracle (keys of the wrong sequence, the
+  query offsets used for the keys, values not offset, heads reversed in O or
+  in lse).
 """
 
 import math
@@ -98,3 +100,36 @@ def test_bad_offsets_rejected():
         oracle.attention_varlen_ref(q, k, v, [0, 3, 2], cu_k, 1.0)
     with pytest.raises(ValueError):
         oracle.attention_varlen_ref(q, k, v, [0, 2, 5], cu_k, 1.0)
+
+
+PLANTED = {
+    "keys_of_previous_sequence": ("ka, kb = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]",
+                                  "ka, kb = cu_q[b], cu_q[b + 1], cu_k[max(b - 1, 0)], cu_k[max(b, 1)]"),
+    "query_offsets_for_keys": ("ks = k[ka:kb]", "ks = k[qa:qa + (kb - ka)]"),
+    "values_from_the_start": ("vs = v[ka:kb]", "vs = v[:kb - ka]"),
+    "heads_reversed": ("o[qa:qb] = ob[0].transpose(1, 0, 2)",
+                       "o[qa:qb] = ob[0][::-1].transpose(1, 0, 2)"),
+    "lse_heads_reversed": ("lse[:, qa:qb] = lb[0]", "lse[:, qa:qb] = lb[0][::-1]"),
+}
+
+
+@pytest.mark.parametrize("kind", sorted(PLANTED))
+def test_planted_varlen_mistakes_are_caught(kind, monkeypatch):
+    import inspect
+
+    from oracle import varlen as varlen_mod
+
+    old, new = PLANTED[kind]
+    src = inspect.getsource(varlen_mod.attention_varlen_ref)
+    assert src.count(old) == 1, old
+    ns = dict(vars(varlen_mod))
+    exec(compile(src.replace(old, new), varlen_mod.__file__, "exec"), ns)
+    monkeypatch.setattr(oracle, "attention_varlen_ref", ns["attention_varlen_ref"])
+    failed = 0
+    for lq, lk in CASES:
+        for causal in (False, True):
+            try:
+                test_varlen_matches_brute_force(lq, lk, causal)
+            except (AssertionError, ValueError):
+                failed += 1
+    assert failed > 0, f"no pin caught the planted mistake {kind!r}"
