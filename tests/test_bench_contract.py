@@ -7,6 +7,8 @@
 * Under a multi-rank launch the reference arm runs on rank 0 alone; the other
   ranks exit 0 without work or output.
 * Argument checks: at least 3 warm-up steps; the reference arm is forward only.
+* The kernel-source hash that ties the committed DRAM counters to the code
+  ignores comments and whitespace and changes with any code edit.
 """
 
 import json
@@ -76,3 +78,25 @@ def test_argument_checks():
     assert r.returncode != 0 and "--warmup must be >= 3" in r.stderr
     r = _run("--impl", "reference", "--pass", "bwd", timeout=120)
     assert r.returncode != 0 and "forward oracle only" in r.stderr
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path):
+    """The committed DRAM counters stay attached to the kernel across comment
+    edits and are dropped by any code change."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    base = "__global__ void k(int* p) {\n  p[0] = 1;  // store\n}\n"
+    variants = {
+        "same": base,
+        "comments": "/* header\n   text */\n__global__ void k(int* p) {\n  // new note\n  p[0] = 1;\n}\n",
+        "spacing": "__global__   void k(int* p)\n{ p[0] = 1; }",
+        "code": "__global__ void k(int* p) {\n  p[0] = 2;  // store\n}\n",
+    }
+    hashes = {}
+    for name, text in variants.items():
+        f = tmp_path / f"{name}.cuh"
+        f.write_text(text)
+        hashes[name] = bench.kernel_hash((str(f),))
+    assert hashes["same"] == hashes["comments"] == hashes["spacing"]
+    assert hashes["code"] != hashes["same"]
