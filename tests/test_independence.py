@@ -38,3 +38,22 @@ def test_product_never_imports_the_oracle():
             if fn.endswith((".cu", ".cuh", ".h", ".cpp")):
                 text = open(os.path.join(base, fn), encoding="utf-8").read()
                 assert "oracle" not in text.lower(), fn
+
+
+def test_bench_reaches_the_oracle_only_from_its_cpu_legs():
+    """bench.py imports the oracle only inside the functions that time it on
+    the host (the CPU baseline and the reference arm's oracle samples), never
+    at module level or on the GPU path."""
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py"), encoding="utf-8").read())
+    allowed = {"oracle_sample", "bwd_oracle_sample", "cpu_baseline"}
+
+    def visit(node, func):
+        for child in ast.iter_child_nodes(node):
+            name = child.name if isinstance(child, (ast.FunctionDef, ast.AsyncFunctionDef)) else func
+            if isinstance(child, ast.Import) and any(a.name.split(".")[0] == "oracle" for a in child.names):
+                assert name in allowed, f"bench.py imports the oracle in {name!r} (line {child.lineno})"
+            if isinstance(child, ast.ImportFrom) and (child.module or "").split(".")[0] == "oracle":
+                assert name in allowed, f"bench.py imports the oracle in {name!r} (line {child.lineno})"
+            visit(child, name)
+
+    visit(tree, None)
