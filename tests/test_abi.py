@@ -189,3 +189,16 @@ def test_binding_signatures_match_the_headers():
         assert len(args) == len(params), (name, len(args), len(params))
         for i, (got, want) in enumerate(zip(args, params)):
             assert got is _ctype_of(want), (name, i, want)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No CPU fallback: without the built library every entry point raises."""
+    monkeypatch.setattr(fa, "_LIB", None)
+    monkeypatch.setattr(fa, "library_path", lambda: str(tmp_path / "libfa_b200.so"))
+    p = 1 << 20
+    for call in (lambda: fa.fa_fwd(p, p, p, p, p, 1, 1, 128, 64, 0.125, 0, None),
+                 lambda: fa.fa_bwd_workspace_bytes(1, 1, 128),
+                 lambda: fa.fa_status_string(0),
+                 fa.load_library):
+        with pytest.raises(FileNotFoundError, match="build it"):
+            call()
