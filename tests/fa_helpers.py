@@ -2,6 +2,8 @@
 compare with the float64 oracle on the same seeded bf16 inputs."""
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import torch
@@ -63,19 +65,37 @@ def full_parity(q, k, v, causal=False, mask=None, scale=None):
     return assert_parity(o, lse, o_ref, lse_ref)
 
 
-def sample_rows(B, H, N, count, seed, per_tile=True):
-    """(b, h, i) samples: first and last rows, tile edges, one random row in
-    every (b, h, 128-row query tile) when `per_tile`, and random rows up to
-    `count` extra."""
-    r = np.random.default_rng(seed)
-    rows = {(0, 0, 0), (B - 1, H - 1, N - 1), (0, H - 1, min(N - 1, 127)),
-            (B - 1, 0, min(N - 1, 128)), (0, 0, N // 2)}
-    if per_tile:
-        for b in range(B):
-            for h in range(H):
-                for t0 in range(0, N, 128):
-                    rows.add((b, h, int(r.integers(t0, min(N, t0 + 128)))))
-    target = len(rows) + count
-    while len(rows) < target:
-        rows.add((int(r.integers(B)), int(r.integers(H)), int(r.integers(N))))
-    return sorted(rows)
+def _pool_size():
+    return max(1, min(16, os.cpu_count() or 1))
+
+
+def oracle_per_head(fn, heads):
+    """Run `fn(b, h)` for every (b, h) in `heads` on a thread pool (NumPy
+    releases the GIL in its array loops and BLAS calls, so the heads run side
+    by side), the host's cores shared out between the tasks as BLAS threads.
+    Returns the results in order."""
+    from threadpoolctl import threadpool_limits
+
+    workers = min(_pool_size(), len(heads))
+    with threadpool_limits(max(1, (os.cpu_count() or 1) // workers)), ThreadPoolExecutor(workers) as ex:
+        return list(ex.map(lambda bh: fn(*bh), heads))
+
+
+def oracle_full(q, k, v, scale, causal=False, mask=None):
+    """The float64 oracle on every row of every head (numpy inputs), one
+    thread-pool task per head.  Same function, same arithmetic as calling
+    oracle.attention_ref on the whole batch."""
+    B, H, N, _ = q.shape
+    heads = [(b, h) for b in range(B) for h in range(H)]
+
+    def one(b, h):
+        bm = None if mask is None else mask[b:b + 1, h:h + 1]
+        return oracle.attention_ref(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1],
+                                    scale, causal=causal, block_mask=bm)
+
+    res = oracle_per_head(one, heads)
+    o = np.empty((B, H, N, v.shape[-1]))
+    lse = np.empty((B, H, N))
+    for (b, h), (oh, lh) in zip(heads, res):
+        o[b, h], lse[b, h] = oh[0, 0], lh[0, 0]
+    return o, lse

@@ -16,8 +16,8 @@ import torch
 
 import exact_attention_120_b200 as fa
 import oracle
-from exact_attention_120_b200.workloads import make_qkv
-from fa_helpers import to_np64
+from exact_attention_120_b200.workloads import WORKLOADS, make_inputs, make_qkv
+from fa_helpers import oracle_per_head, to_np64
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
@@ -78,3 +78,35 @@ def test_bwd_block_sparse():
 
 def test_bwd_longer_sequence():
     _check(*_case(1, 4, 2048, 2048, 128, seed=41), True)
+
+
+def test_bwd_long_full_shape_two_heads_every_row():
+    # The backward in the configuration bench.py --pass bwd times: the long
+    # full-attention workload (B=1, H=16, N=16384, d=128, Q/K std 3) with the
+    # bench's seeded dO, on all 16 heads.  Heads 0 and 15 are compared with the
+    # float64 gradient oracle on every row of dQ, dK and dV.
+    w = WORKLOADS["long_full"]
+    q, k, v, _ = make_inputs(w)
+    g = torch.Generator().manual_seed(w.seed + 7)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), do.to(DEV)
+    o, lse = fa.attention_forward(qd, kd, vd)
+    dq, dk, dv = fa.attention_backward(qd, kd, vd, o, lse, dod)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(None) == fa.FA_OK
+    heads = [(0, 0), (0, w.H - 1)]
+    got = [tuple(to_np64(t[b, h]) for t in (dq, dk, dv)) for b, h in heads]
+    del qd, kd, vd, dod, o, lse, dq, dk, dv
+
+    def one(b, h):
+        sl = lambda t: to_np64(t[b:b + 1, h:h + 1])  # noqa: E731
+        return oracle.attention_bwd_ref(sl(q), sl(k), sl(v), sl(do), w.scale)
+
+    refs = oracle_per_head(one, heads)
+    for (b, h), g3, r3 in zip(heads, got, refs):
+        for name, gt, want in zip(("dq", "dk", "dv"), g3, r3):
+            want = want[0, 0]
+            assert np.all(np.isfinite(gt)), (name, h)
+            err = np.max(np.abs(gt - want))
+            scale = max(np.max(np.abs(want)), 1e-6)
+            assert err <= REL * scale, f"head {h} {name}: max|d| {err:.3e} > {REL} x {scale:.3e}"

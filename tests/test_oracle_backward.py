@@ -61,14 +61,17 @@ def test_gradients_match_finite_differences(mode, nq, nk):
         np.testing.assert_allclose(g, num, rtol=1e-5, atol=1e-7, err_msg=name)
 
 
+@pytest.mark.parametrize("row_chunk", [1024, 5])
 @pytest.mark.parametrize("nq,nk,causal", [(16, 16, False), (16, 16, True), (8, 20, True),
                                           (20, 9, False)])
-def test_gradients_match_torch_autograd(nq, nk, causal):
+def test_gradients_match_torch_autograd(nq, nk, causal, row_chunk):
+    # row_chunk = 5 cuts the query rows into ragged chunks, so dK and dV are
+    # summed over several chunks.
     from torch.nn.attention.bias import causal_lower_right
 
     B, H, d, scale = 2, 2, 8, 0.35
     q, k, v, do = _case(B, H, nq, nk, d, nq + nk)
-    dq, dk, dv = oracle.attention_bwd_ref(q, k, v, do, scale, causal)
+    dq, dk, dv = oracle.attention_bwd_ref(q, k, v, do, scale, causal, row_chunk=row_chunk)
     tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
     mask = causal_lower_right(nq, nk) if causal else None
     out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=scale)
@@ -109,48 +112,81 @@ def test_invisible_keys_get_no_gradient():
     assert np.abs(dk[:, :, :4]).sum() > 0
 
 
-def test_delta_is_row_dot():
-    o = _r(1).normal(size=(1, 2, 5, 3))
-    do = _r(2).normal(size=(1, 2, 5, 3))
-    np.testing.assert_allclose(oracle.softmax_delta(o, do), np.einsum("bhnd,bhnd->bhn", o, do))
+@pytest.mark.parametrize("causal", [False, True])
+def test_delta_equals_probability_weighted_dp(causal):
+    # D_i = dO_i . O_i must equal sum_j P_ij (dO_i . v_j), with P taken from
+    # the pure-Python brute force's logsumexp (P_ij = exp(s_ij - lse_i)) and
+    # every sum formed with math.fsum: a second route to D that never forms O.
+    B, H, nq, nk, d, scale = 1, 2, 5, 7, 3, 0.8
+    q, k, v, do = _case(B, H, nq, nk, d, 21)
+    o, lse = oracle.attention_brute(q.tolist(), k.tolist(), v.tolist(), scale, causal=causal)
+    o, lse = np.array(o), np.array(lse)
+    got = oracle.softmax_delta(o, do)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nq):
+                terms = []
+                for j in range(nk):
+                    if causal and j > i + (nk - nq):
+                        continue
+                    s_ij = scale * math.fsum(q[b, h, i, t] * k[b, h, j, t] for t in range(d))
+                    dp_ij = math.fsum(do[b, h, i, t] * v[b, h, j, t] for t in range(d))
+                    terms.append(math.exp(s_ij - lse[b, h, i]) * dp_ij)
+                assert abs(got[b, h, i] - math.fsum(terms)) <= 1e-12 * (1 + abs(got[b, h, i]))
 
 
 # Plausible mistakes planted in a copy of the gradient oracle (on the CPU): a
 # dropped or sign-flipped row term, a missing scale, a swapped operand, the
 # mask left out.  Each must make at least one pin above fail.
 PLANTED = {
-    "drop_delta": ("ds = p * (dp - dd[:, None])", "ds = p * dp"),
-    "delta_sign": ("ds = p * (dp - dd[:, None])", "ds = p * (dp + dd[:, None])"),
-    "dq_no_scale": ("dq[b, h] = scale * (ds @ k[b, h])", "dq[b, h] = ds @ k[b, h]"),
-    "dq_uses_v": ("dq[b, h] = scale * (ds @ k[b, h])", "dq[b, h] = scale * (ds @ v[b, h])"),
-    "dv_uses_o": ("dv[b, h] = p.T @ do[b, h]", "dv[b, h] = p.T @ o"),
-    "delta_from_q": ("dd = np.sum(do[b, h] * o, axis=1)", "dd = np.sum(do[b, h] * q[b, h], axis=1)"),
-    "dk_uses_do": ("dk[b, h] = scale * (ds.T @ q[b, h])", "dk[b, h] = scale * (ds.T @ do[b, h])"),
-    "mask_ignored": ("s = np.where(vis, s, -np.inf)", "s = s"),
+    "drop_delta": ("attention_bwd_ref", "ds = p * (dp - dd[:, None])", "ds = p * dp"),
+    "delta_sign": ("attention_bwd_ref", "ds = p * (dp - dd[:, None])", "ds = p * (dp + dd[:, None])"),
+    "dq_no_scale": ("attention_bwd_ref", "dq[b, h, rows] = scale * (ds @ k[b, h])",
+                    "dq[b, h, rows] = ds @ k[b, h]"),
+    "dq_uses_v": ("attention_bwd_ref", "dq[b, h, rows] = scale * (ds @ k[b, h])",
+                  "dq[b, h, rows] = scale * (ds @ v[b, h])"),
+    "dv_uses_o": ("attention_bwd_ref", "dv[b, h] += p.T @ doc", "dv[b, h] += p.T @ o"),
+    "delta_from_q": ("attention_bwd_ref", "dd = softmax_delta(o, doc)", "dd = softmax_delta(qc, doc)"),
+    "dk_uses_do": ("attention_bwd_ref", "dk[b, h] += scale * (ds.T @ qc)",
+                   "dk[b, h] += scale * (ds.T @ doc)"),
+    "mask_ignored": ("attention_bwd_ref", "s = np.where(vis, s, -np.inf)", "s = s"),
+    "dk_last_chunk_only": ("attention_bwd_ref", "dk[b, h] += scale * (ds.T @ qc)",
+                           "dk[b, h] = scale * (ds.T @ qc)"),
+    "delta_squares_o": ("softmax_delta", "np.sum(_as64(o) * _as64(do), axis=-1)",
+                        "np.sum(_as64(o) * _as64(o), axis=-1)"),
+    "delta_negated": ("softmax_delta", "np.sum(_as64(o) * _as64(do), axis=-1)",
+                      "-np.sum(_as64(o) * _as64(do), axis=-1)"),
 }
 
 
-def _bwd_mutant(old, new):
+def _bwd_mutant(func, old, new, monkeypatch):
+    """Plant `new` in place of `old` in a copy of oracle.backward's `func`;
+    the copied attention_bwd_ref calls the mutated helpers."""
     import inspect
 
     from oracle import backward as bwd_mod
 
-    src = inspect.getsource(bwd_mod.attention_bwd_ref)
-    assert src.count(old) == 1, old
     ns = dict(vars(bwd_mod))
+    src = inspect.getsource(getattr(bwd_mod, func))
+    assert src.count(old) == 1, old
     exec(compile(src.replace(old, new), bwd_mod.__file__, "exec"), ns)
-    return ns["attention_bwd_ref"]
+    if func != "attention_bwd_ref":
+        exec(compile(inspect.getsource(bwd_mod.attention_bwd_ref), bwd_mod.__file__, "exec"), ns)
+        monkeypatch.setattr(oracle, func, ns[func])
+    monkeypatch.setattr(oracle, "attention_bwd_ref", ns["attention_bwd_ref"])
 
 
 @pytest.mark.parametrize("kind", sorted(PLANTED))
 def test_planted_gradient_mistakes_are_caught(kind, monkeypatch):
-    monkeypatch.setattr(oracle, "attention_bwd_ref", _bwd_mutant(*PLANTED[kind]))
+    _bwd_mutant(*PLANTED[kind], monkeypatch)
     pins = [lambda: test_gradients_match_finite_differences("sparse_causal", 3, 6),
             lambda: test_gradients_match_finite_differences("full", 5, 5),
-            lambda: test_gradients_match_torch_autograd(8, 20, True),
+            lambda: test_gradients_match_torch_autograd(8, 20, True, 1024),
+            lambda: test_gradients_match_torch_autograd(20, 9, False, 5),
             test_constant_values_give_no_query_key_gradient,
             lambda: test_softmax_gradient_rows_sum_to_zero("causal"),
-            test_invisible_keys_get_no_gradient]
+            test_invisible_keys_get_no_gradient,
+            lambda: test_delta_equals_probability_weighted_dp(True)]
     failed = 0
     for pin in pins:
         try:
