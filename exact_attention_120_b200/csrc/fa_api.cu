@@ -27,6 +27,13 @@ namespace {
 // Device-side status word (FA_OK or FA_ERR_DEVICE_TIMEOUT), one per device.
 __device__ int g_fa_status = 0;
 
+// Workspace of fa_fwd_splitkv_noalloc: a fixed array in the module's device
+// memory, so that entry point never allocates.  Every device that loads the
+// library holds it until the process exits; all calls on a device share it.
+// In host code the name only stands in for the symbol: its device address is
+// taken with cudaGetSymbolAddress in the once-per-device set-up below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
 thread_local int t_last_cuda_error = 0;
 
 constexpr unsigned long long kWaitTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s per wait
@@ -41,7 +48,8 @@ struct DeviceState {
   std::once_flag once;
   int status = FA_ERR_CUDA;  // result of the set-up
   int num_sms = 0;
-  int* status_word = nullptr;  // device address of g_fa_status
+  int* status_word = nullptr;     // device address of g_fa_status
+  void* noalloc_scratch = nullptr;  // device address of g_noalloc_scratch
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -90,6 +98,12 @@ int setup_device(int dev, DeviceState& st) {
   e = cudaGetSymbolAddress(&sym, g_fa_status);
   if (e != cudaSuccess) return cuda_fail(e);
   st.status_word = static_cast<int*>(sym);
+  // With this device current: the device address of the no-allocation
+  // workspace (loading the module above already reserved the array).
+  sym = nullptr;
+  e = cudaGetSymbolAddress(&sym, g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e);
+  st.noalloc_scratch = sym;
   return FA_OK;
 }
 
@@ -177,35 +191,51 @@ int causal_group(long long bh, long long nk, int d, int elt_bytes) {
   return (int)std::max(1ll, std::min(bh, g));
 }
 
-// Workspace of fa_fwd_splitkv_noalloc: a fixed array in the module's device
-// memory, so that entry point never allocates.  Every device that loads the
-// library holds it until the process exits; all calls on a device share it.
-static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
-
-// Device address of g_noalloc_scratch per device.  In host code the array's
-// name only stands in for the symbol; the address comes from
-// cudaGetSymbolAddress, taken once per device with that device current.
-struct NoallocState {
-  std::once_flag once;
-  int status = FA_ERR_CUDA;
-  void* scratch = nullptr;
-};
-NoallocState g_noalloc[kMaxDevices];
-
 // Bytes of the split-key workspace: fp32 partial O [splits][rows][d] followed
 // by fp32 partial lse [splits][rows].
 size_t splitkv_workspace_bytes(size_t rows, int d, int splits) {
   return (size_t)splits * rows * ((size_t)d + 1) * sizeof(float);
 }
 
-// Validation, descriptors and launch shared by the entry points.
-int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-               int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
-               void* cuda_stream, unsigned long long timeout_ns, int starve_producer,
-               int num_splits = 1, void* workspace = nullptr, size_t workspace_bytes = 0,
-               bool fp8 = false, float q_descale = 1.f, float k_descale = 1.f,
-               float v_descale = 1.f) {
-  // ---- arguments (nothing is launched on error)
+// True if the byte ranges [a, a + na) and [b, b + nb) share a byte.
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return na > 0 && nb > 0 && x < y + nb && y < x + na;
+}
+
+// A buffer and its size in bytes, for the overlap checks.
+struct Span {
+  const void* p;
+  size_t bytes;
+};
+
+// True if any output overlaps any input or another output.  Inputs may
+// overlap each other (they are only read).
+bool outputs_alias(std::initializer_list<Span> outs, std::initializer_list<Span> ins) {
+  for (const Span* o = outs.begin(); o != outs.end(); ++o) {
+    for (const Span& i : ins)
+      if (overlaps(o->p, o->bytes, i.p, i.bytes)) return true;
+    for (const Span* o2 = o + 1; o2 != outs.end(); ++o2)
+      if (overlaps(o->p, o->bytes, o2->p, o2->bytes)) return true;
+  }
+  return false;
+}
+
+// Work decomposition of a forward call, derived from its sizes.
+struct FwdGeom {
+  long long bh = 0, nqt = 0, nkt = 0, npairs = 0;
+  int kt_per_split = 0, splits = 1;
+  size_t rows = 0;       // B * H * Nq
+  size_t workspace = 0;  // split-key workspace bytes (0 for one slice)
+};
+
+// Every check of a forward call that needs no CUDA call: pointers, sizes,
+// scale, causal flag, head dim, alignment, aliasing and the slice count.
+// Fills `g` on success.
+int check_fwd_args(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
+                   int num_splits, bool fp8, float q_descale, float k_descale, float v_descale,
+                   FwdGeom& g) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARGUMENT;
   if (fp8 && !(std::isfinite(q_descale) && q_descale > 0.f && std::isfinite(k_descale) &&
                k_descale > 0.f && std::isfinite(v_descale) && v_descale > 0.f))
@@ -217,29 +247,42 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return FA_ERR_INVALID_ARGUMENT;
-  const long long bh = (long long)B * H;
-  const long long nqt = (Nq + fa::kBM - 1) / fa::kBM;
-  const long long nkt = (Nk + fa::kBN - 1) / fa::kBN;
-  const long long npairs = (nqt + 1) / 2;
-  if (bh > INT32_MAX || bh * npairs > INT32_MAX || (long long)Nq * d * 2 >= (1ll << 40) ||
+  g.bh = (long long)B * H;
+  g.nqt = (Nq + fa::kBM - 1) / fa::kBM;
+  g.nkt = (Nk + fa::kBN - 1) / fa::kBN;
+  g.npairs = (g.nqt + 1) / 2;
+  if (g.bh > INT32_MAX || g.bh * g.npairs > INT32_MAX || (long long)Nq * d * 2 >= (1ll << 40) ||
       (long long)Nk * d * 2 >= (1ll << 40))
     return FA_ERR_UNSUPPORTED;  // 32-bit work indices and TMA stride limits
-  if (o == q || o == k || o == v) return FA_ERR_INVALID_ARGUMENT;
+  g.rows = (size_t)g.bh * Nq;
+  const size_t eb = fp8 ? 1 : 2;
+  const size_t kv_bytes = (size_t)g.bh * Nk * d * eb;
+  const Span ins[] = {{q, g.rows * d * eb}, {k, kv_bytes}, {v, kv_bytes},
+                      {block_mask, block_mask ? (size_t)(g.bh * g.nqt * g.nkt) : 0}};
+  if (outputs_alias({{o, g.rows * d * 2}, {lse, g.rows * sizeof(float)}},
+                    {ins[0], ins[1], ins[2], ins[3]}))
+    return FA_ERR_INVALID_ARGUMENT;
   if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_INVALID_ARGUMENT;
   // Slices of kt_per_split key tiles; the last one is never empty.
-  const int kt_per_split = (int)((nkt + num_splits - 1) / num_splits);
-  const int splits = (int)((nkt + kt_per_split - 1) / kt_per_split);
-  if (bh * npairs * splits > INT32_MAX) return FA_ERR_UNSUPPORTED;
-  const size_t rows = (size_t)bh * Nq;
-  if (splits > 1) {
-    if (!workspace || !aligned(workspace, 16) ||
-        workspace_bytes < splitkv_workspace_bytes(rows, d, splits))
-      return FA_ERR_INVALID_ARGUMENT;
-  }
+  g.kt_per_split = (int)((g.nkt + num_splits - 1) / num_splits);
+  g.splits = (int)((g.nkt + g.kt_per_split - 1) / g.kt_per_split);
+  if (g.bh * g.npairs * g.splits > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  g.workspace = g.splits > 1 ? splitkv_workspace_bytes(g.rows, d, g.splits) : 0;
+  return FA_OK;
+}
 
-  DeviceState* st = nullptr;
-  int rc = get_device_state(&st);
-  if (rc != FA_OK) return rc;
+// Descriptors and launch shared by the forward entry points.  `g` comes from
+// check_fwd_args.  With more than one slice, `workspace` holds at least
+// g.workspace bytes and overlaps none of the call's buffers.
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
+               void* cuda_stream, unsigned long long timeout_ns, int starve_producer,
+               const FwdGeom& g, DeviceState* st, void* workspace = nullptr, bool fp8 = false,
+               float q_descale = 1.f, float k_descale = 1.f, float v_descale = 1.f) {
+  const long long bh = g.bh, nqt = g.nqt, nkt = g.nkt, npairs = g.npairs;
+  const int splits = g.splits, kt_per_split = g.kt_per_split;
+  const size_t rows = g.rows;
+  int rc = FA_OK;
   if (!is_device_pointer(q) || !is_device_pointer(k) || !is_device_pointer(v) ||
       !is_device_pointer(o) || !is_device_pointer(lse) ||
       (block_mask && !is_device_pointer(block_mask)) ||
@@ -307,6 +350,34 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return FA_OK;
 }
 
+// A forward call with a caller workspace (or none): host checks, then the
+// device set-up, then the launch.
+int run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq,
+            int Nk, int d, float scale, int causal, const uint8_t* block_mask, void* cuda_stream,
+            unsigned long long timeout_ns, int starve_producer, int num_splits = 1,
+            void* workspace = nullptr, size_t workspace_bytes = 0, bool fp8 = false,
+            float q_descale = 1.f, float k_descale = 1.f, float v_descale = 1.f) {
+  FwdGeom g;
+  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, num_splits,
+                          fp8, q_descale, k_descale, v_descale, g);
+  if (rc != FA_OK) return rc;
+  if (g.splits > 1) {
+    const size_t eb = fp8 ? 1 : 2;
+    const size_t kv_bytes = (size_t)g.bh * Nk * d * eb;
+    if (!workspace || !aligned(workspace, 16) || workspace_bytes < g.workspace ||
+        outputs_alias({{workspace, g.workspace}},
+                      {{q, g.rows * d * eb}, {k, kv_bytes}, {v, kv_bytes}, {o, g.rows * d * 2},
+                       {lse, g.rows * sizeof(float)},
+                       {block_mask, block_mask ? (size_t)(g.bh * g.nqt * g.nkt) : 0}}))
+      return FA_ERR_INVALID_ARGUMENT;
+  }
+  DeviceState* st = nullptr;
+  if ((rc = get_device_state(&st)) != FA_OK) return rc;
+  return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
+                    timeout_ns, starve_producer, g, st, workspace, fp8, q_descale, k_descale,
+                    v_descale);
+}
+
 }  // namespace
 
 extern "C" {
@@ -314,15 +385,15 @@ extern "C" {
 int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                   int N, int d, float scale, int causal, const uint8_t* block_mask,
                   void* cuda_stream) {
-  return launch_fwd(q, k, v, o, lse, B, H, N, N, d, scale, causal, block_mask, cuda_stream,
-                    kWaitTimeoutNs, 0);
+  return run_fwd(q, k, v, o, lse, B, H, N, N, d, scale, causal, block_mask, cuda_stream,
+                 kWaitTimeoutNs, 0);
 }
 
 int fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
               int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
               void* cuda_stream) {
-  return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
-                    kWaitTimeoutNs, 0);
+  return run_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
+                 kWaitTimeoutNs, 0);
 }
 
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int num_splits) {
@@ -349,36 +420,28 @@ int fa_fwd_splitkv_heuristic(int B, int H, int Nq, int Nk) {
 int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                    int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
                    int num_splits, void* workspace, size_t workspace_bytes, void* cuda_stream) {
-  return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
-                    kWaitTimeoutNs, 0, num_splits, workspace, workspace_bytes);
+  return run_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
+                 kWaitTimeoutNs, 0, num_splits, workspace, workspace_bytes);
 }
 
 int fa_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                            int H, int Nq, int Nk, int d, float scale, int causal,
                            const uint8_t* block_mask, int num_splits, void* cuda_stream) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-  NoallocState& ns = g_noalloc[dev];
-  std::call_once(ns.once, [&] {  // first call on this device: find the array
-    void* ptr = nullptr;
-    const cudaError_t r = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (r != cudaSuccess) {
-      t_last_cuda_error = static_cast<int>(r);
-      ns.status = FA_ERR_CUDA;
-      return;
-    }
-    ns.scratch = ptr;
-    ns.status = FA_OK;
-  });
-  if (ns.status != FA_OK) return ns.status;
-  const size_t need = fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits);
-  if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  // Every host-side check first, with no CUDA call; then the size limit.
+  FwdGeom g;
+  int rc = check_fwd_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, num_splits,
+                          false, 1.f, 1.f, 1.f, g);
+  if (rc != FA_OK) return rc;
+  if (g.workspace > (size_t)FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  // The once-per-device set-up (the first library call on this device) took
+  // the array's device address with this device current.
+  DeviceState* st = nullptr;
+  if ((rc = get_device_state(&st)) != FA_OK) return rc;
   // The split kernel writes every partial it later reads (empty slices
-  // included), so nothing in the array has to start at zero.
+  // included), so nothing in the array has to start at zero.  The array is
+  // the library's own memory: it cannot overlap the caller's buffers.
   return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
-                    kWaitTimeoutNs, 0, num_splits, need > 0 ? ns.scratch : nullptr, need);
+                    kWaitTimeoutNs, 0, g, st, g.splits > 1 ? st->noalloc_scratch : nullptr);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq) {
@@ -405,10 +468,15 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (bh * nqt > INT32_MAX || bh * nkt > INT32_MAX || (long long)Nq * d * 2 >= (1ll << 40) ||
       (long long)Nk * d * 2 >= (1ll << 40))
     return FA_ERR_UNSUPPORTED;
-  if (workspace_bytes < fa_bwd_workspace_bytes(B, H, Nq)) return FA_ERR_INVALID_ARGUMENT;
-  for (const void* out : std::initializer_list<const void*>{dq, dk, dv})
-    if (out == q || out == k || out == v || out == o || out == dout) return FA_ERR_INVALID_ARGUMENT;
-  if (dq == dk || dq == dv || dk == dv) return FA_ERR_INVALID_ARGUMENT;
+  const size_t ws_need = fa_bwd_workspace_bytes(B, H, Nq);
+  if (workspace_bytes < ws_need) return FA_ERR_INVALID_ARGUMENT;
+  {
+    const size_t qb = (size_t)bh * Nq * d * 2, kb = (size_t)bh * Nk * d * 2;
+    if (outputs_alias({{dq, qb}, {dk, kb}, {dv, kb}, {workspace, ws_need}},
+                      {{q, qb}, {k, kb}, {v, kb}, {o, qb}, {lse, (size_t)bh * Nq * sizeof(float)},
+                       {dout, qb}, {block_mask, block_mask ? (size_t)(bh * nqt * nkt) : 0}}))
+      return FA_ERR_INVALID_ARGUMENT;
+  }
 
   DeviceState* st = nullptr;
   int rc = get_device_state(&st);
@@ -466,15 +534,15 @@ int fa_testing_fwd_starved(const void* q, const void* k, const void* v, void* o,
                            const uint8_t* block_mask, void* cuda_stream,
                            unsigned long long timeout_ns) {
   if (timeout_ns == 0 || timeout_ns > kWaitTimeoutNs) return FA_ERR_INVALID_ARGUMENT;
-  return launch_fwd(q, k, v, o, lse, B, H, N, N, d, scale, causal, block_mask, cuda_stream,
-                    timeout_ns, 1);
+  return run_fwd(q, k, v, o, lse, B, H, N, N, d, scale, causal, block_mask, cuda_stream,
+                 timeout_ns, 1);
 }
 
 int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
                float q_descale, float k_descale, float v_descale, void* cuda_stream) {
-  return launch_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
-                    kWaitTimeoutNs, 0, 1, nullptr, 0, true, q_descale, k_descale, v_descale);
+  return run_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, block_mask, cuda_stream,
+                 kWaitTimeoutNs, 0, 1, nullptr, 0, true, q_descale, k_descale, v_descale);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -489,11 +557,17 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
       !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
     return FA_ERR_INVALID_ARGUMENT;
-  if (o == q || o == k || o == v) return FA_ERR_INVALID_ARGUMENT;
   const long long bh = (long long)B * H;
   const long long nqt = (max_seqlen_q + fa::kBM - 1) / fa::kBM;
   const long long npairs = (nqt + 1) / 2;
   if (bh * npairs > INT32_MAX || (long long)total_q * H > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  {
+    const size_t qb = (size_t)total_q * H * d * 2, kb = (size_t)total_k * H * d * 2;
+    const size_t cb = ((size_t)B + 1) * sizeof(int);
+    if (outputs_alias({{o, qb}, {lse, (size_t)total_q * H * sizeof(float)}},
+                      {{q, qb}, {k, kb}, {v, kb}, {cu_seqlens_q, cb}, {cu_seqlens_k, cb}}))
+      return FA_ERR_INVALID_ARGUMENT;
+  }
 
   DeviceState* st = nullptr;
   int rc = get_device_state(&st);

@@ -31,8 +31,11 @@
  * Layouts and types (all buffers are owned by the caller; the library
  * allocates nothing per call and keeps no pointer after the call returns):
  *   q, k, v, o   device memory, bfloat16, contiguous [B, H, N, d] (d fastest),
- *                16-byte aligned.  o may not alias q, k or v.
+ *                16-byte aligned.
  *   lse          device memory, float32, contiguous [B, H, N], 4-byte aligned.
+ *                No byte of o or lse may lie inside q, k, v, block_mask or
+ *                the other output (checked by address range; inputs may
+ *                overlap each other).
  *   block_mask   NULL, or device memory, uint8, contiguous
  *                [B, H, ceil(N/128), ceil(N/128)], 1 (non-zero) = keep.
  *   d            64 or 128.
@@ -45,7 +48,10 @@
  * kernel surfaces at the caller's next synchronisation; a device-side wait
  * that exceeded its time limit is reported by fa_device_status().  No C++
  * exception crosses this interface.  The entry points may be called from
- * several host threads; per-device set-up is done once, under a lock.
+ * several host threads; per-device set-up is done once, under a lock, by the
+ * first call of any entry point on that device (it loads the library's
+ * device code, whose fixed arrays are then reserved; see
+ * fa_fwd_splitkv_noalloc).
  */
 #ifndef FA_B200_FA_H_
 #define FA_B200_FA_H_
@@ -118,7 +124,8 @@ FA_API int fa_fwd_qk(const void* q, const void* k, const void* v, void* o, float
  * workspace: device memory, 16-byte aligned, at least
  *   fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, num_splits) bytes, owned by
  *   the caller and overwritten by the call.  It may be NULL when that size is 0
- *   (a single slice).
+ *   (a single slice); otherwise its first that many bytes may not overlap any
+ *   other buffer of the call.
  * Calls that share one workspace must not overlap on the GPU.  Two launches are
  * enqueued on `cuda_stream` when there is more than one slice.
  */
@@ -148,14 +155,21 @@ FA_API size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d
  * (fa_fwd_splitkv_workspace_bytes(...) > FA_NOALLOC_SCRATCH_BYTES) is rejected
  * with FA_ERR_UNSUPPORTED before anything is launched.
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, once per device, with that device current).  Make that
- * first call before capturing any stream.
+ * The array is reserved when the library's device code is loaded, which the
+ * first call of any entry point on a device does, together with the set-up
+ * that looks up the array's device address (cudaGetSymbolAddress, once per
+ * device, with that device current).  A caller that may not allocate at call
+ * time makes one call at initialisation (fa_device_status is enough), and
+ * that first call comes before any stream capture.  Argument errors are
+ * found before any CUDA call, as for the other entry points.
  *
  * All calls on a device share the one array, and it keeps the last call's
  * contents.  Calls whose kernels overlap on the GPU (on different streams,
  * without ordering between them) race on it and corrupt each other's results:
- * serialise them.  No part of the array needs to start at zero.
+ * serialise them.  No part of the array needs to start at zero.  After a
+ * call whose kernel gave up on a wait (fa_device_status reports
+ * FA_ERR_DEVICE_TIMEOUT), its o and lse are undefined and may hold values
+ * merged from an earlier call's partial results.
  *
  * The pages have no counterpart to this entry point: it is a packaging of
  * fa_fwd_splitkv for callers without an allocator.
@@ -219,7 +233,7 @@ FA_API int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, floa
  *
  * Returns FA_OK, FA_ERR_INVALID_ARGUMENT (null, host or misaligned pointer,
  * B, H, total_q, total_k or max_seqlen_q < 1, bad scale or causal, o
- * aliasing an input), FA_ERR_UNSUPPORTED (d not 64 or 128, no sm_100
+ * or lse overlapping an input or each other), FA_ERR_UNSUPPORTED (d not 64 or 128, no sm_100
  * device, more than 2^31 work units or query rows x H) or FA_ERR_CUDA.
  */
 FA_API int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -236,8 +250,9 @@ FA_API int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, f
  * q, o, dout, dq: bf16 [B, H, Nq, d]; k, v, dk, dv: bf16 [B, H, Nk, d]; lse:
  * fp32 [B, H, Nq] as written by the forward; causal, block_mask, scale and d
  * exactly as passed to the forward (fa_fwd / fa_fwd_qk).  All device memory,
- * 16-byte aligned (lse: 4), owned by the caller; dq, dk, dv must not alias
- * the inputs or each other.
+ * 16-byte aligned (lse: 4), owned by the caller; no byte of dq, dk, dv or
+ * the workspace may lie inside an input or another of them (checked by
+ * address range).
  * workspace: device memory of at least fa_bwd_workspace_bytes(B, H, Nq) bytes,
  *   16-byte aligned, overwritten (it receives D).  Calls sharing a workspace
  *   must not overlap on the GPU.

@@ -67,6 +67,43 @@ def test_argument_errors_before_any_cuda_call(lib):
     assert call(q=p + 8) == fa.FA_ERR_INVALID_ARGUMENT  # not 16-byte aligned
     assert call(o=p) == fa.FA_ERR_INVALID_ARGUMENT      # o aliases q
     assert call(B=1 << 16, H=1 << 16) == fa.FA_ERR_UNSUPPORTED  # B*H beyond 32 bits
+    # Overlap by address range, not only equal pointers (q, k, v are 16 KB
+    # each here; o 16 KB, lse 512 B).
+    assert call(o=p + 4096) == fa.FA_ERR_INVALID_ARGUMENT       # o inside q
+    assert call(o=p * 3 - 4096) == fa.FA_ERR_INVALID_ARGUMENT   # o runs into lse
+    assert call(lse=p + 256) == fa.FA_ERR_INVALID_ARGUMENT      # lse inside q
+    assert call(lse=p * 2 + 16384 - 4) == fa.FA_ERR_INVALID_ARGUMENT  # last float of o
+    assert call(mask=p * 3 + 16) == fa.FA_ERR_INVALID_ARGUMENT  # lse over the mask
+
+
+def test_noalloc_argument_errors_before_any_cuda_call(lib):
+    """fa_fwd_splitkv_noalloc checks its arguments, and its size limit, before
+    any CUDA call (no device is needed to see these statuses)."""
+    p = 1 << 24  # never dereferenced
+    names = ["q", "k", "v", "o", "lse", "B", "H", "Nq", "Nk", "d", "scale", "causal", "mask",
+             "splits", "stream"]
+    base = [p, p * 2, p * 3, p * 4, p * 5, 1, 2, 64, 4096, 128, 0.1, 0, None, 4, None]
+
+    def call(**kw):
+        a = list(base)
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return lib.fa_fwd_splitkv_noalloc(*a)
+
+    for name in ("q", "k", "v", "o", "lse"):
+        assert call(**{name: None}) == fa.FA_ERR_INVALID_ARGUMENT, name
+    assert call(B=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(scale=float("nan")) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(causal=5) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(q=p + 4) == fa.FA_ERR_INVALID_ARGUMENT      # misaligned
+    assert call(o=p * 2 + 64) == fa.FA_ERR_INVALID_ARGUMENT  # o inside k
+    assert call(splits=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(splits=257) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(d=96) == fa.FA_ERR_UNSUPPORTED
+    # a null pointer is an argument error even when the problem is too large
+    assert call(q=None, Nq=1 << 20) == fa.FA_ERR_INVALID_ARGUMENT
+    # beyond the array: 2 slices x 16257 rows x 129 floats > 16 MiB
+    assert call(B=1, H=1, Nq=16257, Nk=256, splits=2) == fa.FA_ERR_UNSUPPORTED
 
 
 def test_splitkv_workspace_size(lib):
@@ -109,6 +146,9 @@ def test_backward_argument_errors_before_any_cuda_call(lib):
     assert call(ws_bytes=100) == fa.FA_ERR_INVALID_ARGUMENT   # below 2*300*4 bytes of D
     assert call(dq=p) == fa.FA_ERR_INVALID_ARGUMENT           # dq aliases q
     assert call(dv=p * 8) == fa.FA_ERR_INVALID_ARGUMENT       # dv aliases dk
+    # by address range: dk (51 KB) starting inside o, the workspace inside dq
+    assert call(dk=p * 4 + 1024) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(ws=p * 7 + 4096) == fa.FA_ERR_INVALID_ARGUMENT
     assert fa.fa_bwd_workspace_bytes(2, 3, 300) == 2 * 3 * 300 * 4
     assert fa.fa_bwd_workspace_bytes(1, 1, 5) == 32          # rounded up to 16 bytes
     assert fa.fa_bwd_workspace_bytes(0, 1, 5) == 0
@@ -132,6 +172,8 @@ def test_varlen_and_fp8_argument_errors_before_any_cuda_call(lib):
     assert vcall(maxq=0) == fa.FA_ERR_INVALID_ARGUMENT
     assert vcall(cu_k=p * 7 + 2) == fa.FA_ERR_INVALID_ARGUMENT  # offsets not 4-byte aligned
     assert vcall(o=p * 2) == fa.FA_ERR_INVALID_ARGUMENT         # o aliases k
+    assert vcall(lse=p + 512) == fa.FA_ERR_INVALID_ARGUMENT     # lse inside q
+    assert vcall(o=p * 6 - 64) == fa.FA_ERR_INVALID_ARGUMENT    # o runs into cu_seqlens_q
     assert vcall(d=32) == fa.FA_ERR_UNSUPPORTED
     # fa_fwd_fp8(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, mask, qd, kd, vd, stream)
     fbase = [p, p * 2, p * 3, p * 4, p * 5, 1, 1, 128, 128, 128, 0.1, 0, None, 1.0, 1.0, 1.0, None]
