@@ -65,8 +65,17 @@ def full_parity(q, k, v, causal=False, mask=None, scale=None):
     return assert_parity(o, lse, o_ref, lse_ref)
 
 
+def host_cores():
+    """Cores this process may run on (the affinity mask; a container may
+    see far more cores in os.cpu_count() than it is allowed to use)."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except (AttributeError, OSError):
+        return max(1, os.cpu_count() or 1)
+
+
 def _pool_size():
-    return max(1, min(16, os.cpu_count() or 1))
+    return min(16, host_cores())
 
 
 def oracle_per_head(fn, heads):
@@ -77,7 +86,7 @@ def oracle_per_head(fn, heads):
     from threadpoolctl import threadpool_limits
 
     workers = min(_pool_size(), len(heads))
-    with threadpool_limits(max(1, (os.cpu_count() or 1) // workers)), ThreadPoolExecutor(workers) as ex:
+    with threadpool_limits(max(1, host_cores() // workers)), ThreadPoolExecutor(workers) as ex:
         return list(ex.map(lambda bh: fn(*bh), heads))
 
 
