@@ -242,7 +242,7 @@ def run_reference(args, info):
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    emit(info, line)
     return 0
 
 
@@ -580,6 +580,42 @@ def varlen_config(w, job, world):
                   % (job.algorithmic_bytes() // 2**20)}
 
 
+class EventTimer:
+    """CUDA events on the launching stream (and the clock sampler, if any,
+    running from start to stop)."""
+
+    def __init__(self, torch, stream, sampler=None):
+        self.stream, self.sampler = stream, sampler
+        self.e0 = torch.cuda.Event(enable_timing=True)
+        self.e1 = torch.cuda.Event(enable_timing=True)
+
+    def start(self):
+        if self.sampler is not None:
+            self.sampler.start()
+        self.e0.record(self.stream)
+
+    def stop(self):
+        self.e1.record(self.stream)
+
+    def elapsed_ms(self):  # after a synchronise
+        if self.sampler is not None:
+            self.sampler.stop()
+        return self.e0.elapsed_time(self.e1)
+
+
+def rank_workload(w, info):
+    """The workload rank `info.rank` runs: the same shape, its own seed."""
+    return dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank))
+
+
+def emit(info, line, file=None):
+    """Print the JSON line on rank 0 only; returns whether it printed."""
+    if not info.is_root:
+        return False
+    print(json.dumps(line), file=file or sys.stdout, flush=True)
+    return True
+
+
 def run_ours(args, info):
     import torch
 
@@ -595,16 +631,13 @@ def run_ours(args, info):
     stream = torch.cuda.current_stream(dev)
     if args.pass_ == "fp8":
         w = WORKLOADS[args.workload]
-        job = Fp8Job(fa, torch, dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank)),
-                     dev, stream)
+        job = Fp8Job(fa, torch, rank_workload(w, info), dev, stream)
     elif args.pass_ == "varlen":
         w = VARLEN_WORKLOADS["varlen_mix"]
-        job = VarlenJob(fa, torch, dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank)),
-                        dev, stream)
+        job = VarlenJob(fa, torch, rank_workload(w, info), dev, stream)
     else:
         w = WORKLOADS[args.workload]
-        wr = dataclasses.replace(w, seed=sharding.rank_seed(w.seed, info.rank))
-        q, k, v, mask = make_inputs(wr)
+        q, k, v, mask = make_inputs(rank_workload(w, info))
         job = (BwdJob if args.pass_ == "bwd" else FwdJob)(fa, torch, w, q, k, v, mask, dev, stream)
     flops = job.flops
 
@@ -617,20 +650,8 @@ def run_ours(args, info):
 
     # ---- device-timed region: K steps, inputs resident in HBM
     sampler = ClockSampler(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sharding.barrier(dev)
-    torch.cuda.synchronize(dev)
-    sampler.start()
-    e0.record(stream)
-    for _ in range(args.steps):
-        job.launch()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    sampler.stop()
-    sharding.barrier(dev)
-    ms = e0.elapsed_time(e1)
-    ms_max = sharding.max_over_ranks(ms, dev)
-    ms_step = ms_max / args.steps
+    sync = lambda: torch.cuda.synchronize(dev)  # noqa: E731
+    ms_step = sharding.timed_region(job.launch, args.steps, EventTimer(torch, stream, sampler), dev, sync)
     st = fa.fa_device_status(stream.cuda_stream)
     if st != fa.FA_OK:
         raise fa.FaError(st, "device status after timed region")
@@ -652,14 +673,7 @@ def run_ours(args, info):
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(min(3, args.warmup)):
         job.e2e_step()
-    torch.cuda.synchronize(dev)
-    sharding.barrier(dev)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        job.e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = sharding.max_over_ranks(e0.elapsed_time(e1), dev) / e2e_steps
+    e2e_ms = sharding.timed_region(job.e2e_step, e2e_steps, EventTimer(torch, stream), dev, sync)
 
     clocks = sampler.summary()
     if info.world_size > 1:
@@ -713,7 +727,7 @@ def run_ours(args, info):
         line["parity_sample"] = job.parity
     if job.name == "bwd":
         line["config"]["pass"] = "backward (fa_bwd: dQ kernel then dK/dV kernel)"
-    print(json.dumps(line), flush=True)
+    emit(info, line)
     return 0
 
 

@@ -3,8 +3,9 @@
 Attention heads are independent problems: a forward pass has no exchange
 step, so ranks never communicate on the data path.  With N ranks (one
 process per GPU, launched by torchrun), rank r processes its own batch
-slice; the only collectives are a barrier around the timed region and a max
-over ranks of the elapsed device time.
+slice of the workload's shape (its own seed, ``rank_seed``: weak scaling);
+the only collectives are barriers around the timed region and a max over
+ranks of the elapsed time (``timed_region``).
 """
 
 from __future__ import annotations
@@ -29,16 +30,6 @@ def rank_info_from_env(env=None) -> RankInfo:
     env = os.environ if env is None else env
     return RankInfo(int(env.get("RANK", 0)), int(env.get("WORLD_SIZE", 1)),
                     int(env.get("LOCAL_RANK", env.get("RANK", 0))))
-
-
-def shard_units(total_units: int, world_size: int, rank: int) -> range:
-    """Contiguous, balanced split of `total_units` independent units
-    (e.g. (batch, head) problems) over ranks; sizes differ by at most one."""
-    if world_size < 1 or not 0 <= rank < world_size:
-        raise ValueError("bad rank/world size")
-    base, extra = divmod(total_units, world_size)
-    start = rank * base + min(rank, extra)
-    return range(start, start + base + (1 if rank < extra else 0))
 
 
 def rank_seed(seed: int, rank: int) -> int:
@@ -66,6 +57,27 @@ def max_over_ranks(value: float, device=None) -> float:
     t = torch.tensor([float(value)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def timed_region(step, steps: int, timer, device=None, sync=None) -> float:
+    """Time `steps` calls of `step` on every rank and return the job's time
+    per step in ms: the max over ranks.
+
+    Each rank: barrier, `sync()` (e.g. a device synchronise), `timer.start()`,
+    the steps, `timer.stop()`, `sync()`, barrier; then the elapsed time
+    (`timer.elapsed_ms()`) goes through one max-reduction.  Every rank takes
+    the same collective steps in the same order."""
+    barrier(device)
+    if sync is not None:
+        sync()
+    timer.start()
+    for _ in range(steps):
+        step()
+    timer.stop()
+    if sync is not None:
+        sync()
+    barrier(device)
+    return max_over_ranks(timer.elapsed_ms(), device) / steps
 
 
 def barrier(device=None):
