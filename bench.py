@@ -668,6 +668,15 @@ def run_ours(args, info):
     per_ms = sorted(a.elapsed_time(b) for a, b in per)
     pct = lambda f: per_ms[min(len(per_ms) - 1, int(f * len(per_ms)))]  # noqa: E731
 
+    # ---- host side of one call (argument checks, pointer queries, tensor-map
+    # encoding, launch), the device work left running: median of 50 calls
+    host_us = []
+    for _ in range(50):
+        t0 = time.perf_counter()
+        job.launch()
+        host_us.append(1e6 * (time.perf_counter() - t0))
+    torch.cuda.synchronize(dev)
+
     # ---- end to end: pinned host inputs -> device -> public API -> host outputs
     h2d, d2h = job.host_buffers()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -716,6 +725,7 @@ def run_ours(args, info):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "ms_per_step_percentiles": {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9),
                                     "steps": len(per_ms)},
+        "host_us_per_call": statistics.median(host_us),
         "gpu_launches": args.steps * job.launches_per_step,
         "clocks": clocks,
         "cpu_baseline": cpu,

@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     // ------------------------------------------------------ TMA producer ---
     uint32_t it = 0, nu = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+    for (int k = 0, w = unit_of_round(0); w < items && ok; w = unit_of_round(++k)) {
       const BwdUnit<kDQ> u(p, w);
       if constexpr (!kDQ) {
         ok = bwd_wait(bars.ab_empty(), (nu & 1u) ^ 1u, abort_flag, p);
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
       }
       __syncwarp();
     };
-    for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+    for (int k = 0, w = unit_of_round(0); w < items && ok; w = unit_of_round(++k)) {
       const BwdUnit<kDQ> u(p, w);
       ok = bwd_wait(bars.ab_full(), nu & 1u, abort_flag, p);
       if (!ok) break;
@@ -431,7 +431,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
     const float c = p.scale_log2;
     uint32_t sw = 0, it = 0, nu = 0;
     bool ok = true;
-    for (int w = blockIdx.x; w < items && ok; w += gridDim.x) {
+    for (int k = 0, w = unit_of_round(0); w < items && ok; w = unit_of_round(++k)) {
       const BwdUnit<kDQ> u(p, w);
       const int row = u.t * kBM + r;  // query row (kDQ) or key row
       float nlse2 = -INFINITY, delta = 0.f;
