@@ -184,10 +184,15 @@ int encode_varlen_map(CUtensorMap* map, const void* ptr, int T, int H, int d) {
 constexpr int kMaxSplits = 256;
 
 // Heads per group of the causal work order: as many as keep their K and V
-// (2 x nk x d x elt_bytes each) within ~96 MB of the 126 MB L2.
-int causal_group(long long bh, long long nk, int d, int elt_bytes) {
+// (2 x nk x d x elt_bytes each) within `budget_mb` of the 126 MB L2.  Dense
+// batches use 96 MB: their heads all have the longest rows, and splitting
+// them into more groups leaves a tail (mid-size causal: 1043 -> 855 TFLOP/s
+// at 48 MB).  Variable-length batches use 48 MB: there the K/V of the long
+// sequences were read from DRAM about four times over at 96 MB, and 48 MB
+// measured 815 -> 889 TFLOP/s on a mix of 32 sequences.
+int causal_group(long long bh, long long nk, int d, int elt_bytes, long long budget_mb = 96) {
   const long long kv = 2ll * std::max(nk, 1ll) * d * elt_bytes;
-  const long long g = (96ll << 20) / kv;
+  const long long g = (budget_mb << 20) / kv;
   return (int)std::max(1ll, std::min(bh, g));
 }
 
@@ -594,7 +599,7 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   p.bh = (int)bh;
   // Sequences are at most max_seqlen_q long; keys of the longest are bounded
   // by total_k, so group by the query bound (the usual self-attention case).
-  p.group = causal_group(bh, std::min<long long>(max_seqlen_q, total_k), d, 2);
+  p.group = causal_group(bh, std::min<long long>(max_seqlen_q, total_k), d, 2, 48);
   p.items = (int)(bh * npairs);
   p.splits = 1;
   p.kt_per_split = p.nkt;
