@@ -232,6 +232,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   const int lane = threadIdx.x & 31;
   const int items = p.bh * (kDQ ? p.nqt : p.nkt);
 
+  // The next attention launch on the stream may start its prologue now.
+  ptx::launch_dependents();
   if (threadIdx.x == 0) {
     // dQ: both elementwise warpgroups arrive once Q and dO are in tensor
     // memory; dK/dV: the producer's expect-tx arrival for the K, V tiles.
@@ -268,6 +270,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_kernel(const __grid_con
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Everything above is this CTA's prologue; global memory is touched only
+  // after the previous grid on the stream has finished (launch overlap).
+  ptx::grid_dependency_wait();
   const CUtensorMap* mapA = kDQ ? &p.tm_q : &p.tm_k;
   const CUtensorMap* mapB = kDQ ? &p.tm_do : &p.tm_v;
   const CUtensorMap* mapX = kDQ ? &p.tm_k : &p.tm_q;

@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(256) fa_combine_kernel(const float* __restrict
                                                          float* __restrict__ lse, long long rows,
                                                          int splits) {
   constexpr int kCols = D / 32;  // columns per lane: 4 (d=128) or 2 (d=64)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials of the split launch
   const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;

@@ -536,6 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
+  // The next attention launch on the stream may start its prologue now.
+  ptx::launch_dependents();
   if (threadIdx.x == 0) {
     ptx::mbar_init(bQFull, 1);
     ptx::mbar_init(bQEmpty, 1);
@@ -570,6 +572,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Everything above is this CTA's prologue; global memory is touched only
+  // after the previous grid on the stream has finished (launch overlap).
+  ptx::grid_dependency_wait();
 
   if (warp == kLoadWarp) {
     // ------------------------------------------------------ TMA producer ---

@@ -82,6 +82,22 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ------------------------------------------------------- launch overlap ---
+
+// Programmatic dependent launch: the next kernel launched on the stream with
+// the programmatic-serialization attribute may start once every CTA of this
+// grid has executed launch_dependents (or exited); grid_dependency_wait
+// blocks until the previous grid on the stream has completed and its memory
+// operations are visible.  A kernel that waits before its first global
+// memory access overlaps only its prologue with the previous grid's tail.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ TMA ---
 
 // 3-D tiled bulk tensor load global -> shared, completion counted on `bar`.
