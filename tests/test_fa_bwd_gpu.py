@@ -110,3 +110,36 @@ def test_bwd_long_full_shape_two_heads_every_row():
             err = np.max(np.abs(gt - want))
             scale = max(np.max(np.abs(want)), 1e-6)
             assert err <= REL * scale, f"head {h} {name}: max|d| {err:.3e} > {REL} x {scale:.3e}"
+
+
+@pytest.mark.parametrize("name", ["mid_causal", "sparse"])
+def test_bwd_bench_shapes_two_heads_every_row(name):
+    # The backward of the causal and block-sparse workloads in the
+    # configuration bench.py --pass bwd --workload NAME times (all heads, the
+    # bench's seeded dO); two heads compared on every row of dQ, dK and dV.
+    w = WORKLOADS[name]
+    q, k, v, mask = make_inputs(w)
+    g = torch.Generator().manual_seed(w.seed + 7)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = q.to(DEV), k.to(DEV), v.to(DEV), do.to(DEV)
+    md = None if mask is None else mask.to(DEV)
+    o, lse = fa.attention_forward(qd, kd, vd, causal=w.causal, block_mask=md)
+    dq, dk, dv = fa.attention_backward(qd, kd, vd, o, lse, dod, causal=w.causal, block_mask=md)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(None) == fa.FA_OK
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
+    got = [tuple(to_np64(t[b, h]) for t in (dq, dk, dv)) for b, h in heads]
+
+    def one(b, h):
+        sl = lambda t: to_np64(t[b:b + 1, h:h + 1])  # noqa: E731
+        bm = None if mask is None else mask[b:b + 1, h:h + 1].numpy()
+        return oracle.attention_bwd_ref(sl(q), sl(k), sl(v), sl(do), w.scale, causal=w.causal, block_mask=bm)
+
+    refs = oracle_per_head(one, heads)
+    for (b, h), g3, r3 in zip(heads, got, refs):
+        for gname, gt, want in zip(("dq", "dk", "dv"), g3, r3):
+            want = want[0, 0]
+            assert np.all(np.isfinite(gt)), (gname, b, h)
+            err = np.max(np.abs(gt - want))
+            scale = max(np.max(np.abs(want)), 1e-6)
+            assert err <= REL * scale, f"({b},{h}) {gname}: max|d| {err:.3e} > {REL} x {scale:.3e}"
