@@ -78,10 +78,10 @@ int setup_device(int dev, DeviceState& st) {
                              fa::Cfg<128, true>::kSmemBytes);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(fa::fa_fwd_kernel<fa::Cfg<64>, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fa::Cfg<64>::kSmemBytes);
+                             fa::fwd_smem_bytes<fa::Cfg<64>, true>());
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(fa::fa_fwd_kernel<fa::Cfg<128>, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fa::Cfg<128>::kSmemBytes);
+                             fa::fwd_smem_bytes<fa::Cfg<128>, true>());
   if (e != cudaSuccess) return cuda_fail(e);
   e = cudaFuncSetAttribute(fa::fa_bwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            fa::BwdCfg<64>::kSmemBytes);
@@ -614,9 +614,6 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
 
   fa::KernelParams p;
   std::memset(&p, 0, sizeof(p));
-  if ((rc = encode_varlen_map(&p.tm_q, q, total_q, H, d)) != FA_OK) return rc;
-  if ((rc = encode_varlen_map(&p.tm_k, k, total_k, H, d)) != FA_OK) return rc;
-  if ((rc = encode_varlen_map(&p.tm_v, v, total_k, H, d)) != FA_OK) return rc;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.o_v8 = aligned(o, 32) ? 1 : 0;
   p.lse = lse;
@@ -627,11 +624,6 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   p.nkt = (total_k + fa::kBN - 1) / fa::kBN;
   p.causal_off = 0;
   p.npairs = (int)npairs;
-  p.bh = (int)bh;
-  // Sequences are at most max_seqlen_q long; keys of the longest are bounded
-  // by total_k, so group by the query bound (the usual self-attention case).
-  p.group = causal_group(bh, std::min<long long>(max_seqlen_q, total_k), d, 2, 48);
-  p.items = (int)(bh * npairs);
   p.splits = 1;
   p.kt_per_split = p.nkt;
   p.causal = causal;
@@ -639,21 +631,38 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
   p.o_scale = 1.0f;
   p.timeout_ns = kWaitTimeoutNs;
   p.status = st->status_word;
-  p.cu_q = cu_seqlens_q;
-  p.cu_k = cu_seqlens_k;
   p.heads = H;
   p.total_q = total_q;
   p.total_k = total_k;
-
-  const int grid = p.items < st->num_sms ? p.items : st->num_sms;
+  // Causal order: the heads of one sequence are taken in groups whose K/V
+  // together fill at most 48 MiB of L2.
+  p.group_keys = (int)((48ll << 20) / (2ll * d * 2));
+  if ((rc = encode_varlen_map(&p.tm_q, q, total_q, H, d)) != FA_OK) return rc;
+  if ((rc = encode_varlen_map(&p.tm_k, k, total_k, H, d)) != FA_OK) return rc;
+  if ((rc = encode_varlen_map(&p.tm_v, v, total_k, H, d)) != FA_OK) return rc;
+  // One launch per fa::kMaxVarlenSeqs sequences (the kernel's table of their
+  // first work units); the offsets are absolute, so a later launch only
+  // starts further into cu_seqlens.  The kernel deals the units that exist;
+  // the grid is sized by the bound max_seqlen_q gives.
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-  const bool overlap = p.items <= 2 * st->num_sms;
-  cudaError_t e;
-  if (d == 64)
-    e = launch(overlap, fa::fa_fwd_kernel<fa::Cfg<64>, true>, grid, fa::kThreads, fa::Cfg<64>::kSmemBytes, stream, p);
-  else
-    e = launch(overlap, fa::fa_fwd_kernel<fa::Cfg<128>, true>, grid, fa::kThreads, fa::Cfg<128>::kSmemBytes, stream, p);
-  if (e != cudaSuccess) return cuda_fail(e);
+  for (int b0 = 0; b0 < B; b0 += fa::kMaxVarlenSeqs) {
+    const int nseq = std::min(B - b0, fa::kMaxVarlenSeqs);
+    p.cu_q = cu_seqlens_q + b0;
+    p.cu_k = cu_seqlens_k + b0;
+    p.nseq = nseq;
+    p.bh = nseq * H;
+    p.items = (int)(p.bh * npairs);
+    const int grid = p.items < st->num_sms ? p.items : st->num_sms;
+    const bool overlap = p.items <= 2 * st->num_sms;
+    cudaError_t e;
+    if (d == 64)
+      e = launch(overlap, fa::fa_fwd_kernel<fa::Cfg<64>, true>, grid, fa::kThreads,
+                 fa::fwd_smem_bytes<fa::Cfg<64>, true>(), stream, p);
+    else
+      e = launch(overlap, fa::fa_fwd_kernel<fa::Cfg<128>, true>, grid, fa::kThreads,
+                 fa::fwd_smem_bytes<fa::Cfg<128>, true>(), stream, p);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   return FA_OK;
 }
 

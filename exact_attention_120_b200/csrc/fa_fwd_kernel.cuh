@@ -66,6 +66,9 @@ constexpr int kLoadWarp = 1;
 constexpr int kFirstSoftmaxWarp = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kStatusTimeout = 4;  // == FA_ERR_DEVICE_TIMEOUT
+// Variable-length batches: sequences per launch, bounded by the shared-memory
+// table of their first work units (larger batches take several launches).
+constexpr int kMaxVarlenSeqs = 4096;
 
 struct KernelParams {
   CUtensorMap tm_q;  // 3-D maps over [B*H][N][D] bf16, box 64 x 128 x 1, 128B swizzle
@@ -111,6 +114,8 @@ struct KernelParams {
   int heads;
   int total_q;
   int total_k;
+  int nseq;        // sequences of this launch (at most kMaxVarlenSeqs)
+  int group_keys;  // causal order: keys whose K/V of one head fit the L2 share of a head group
 };
 
 // Sizes of the (b, h) problem a work unit belongs to.  Dense batches: every
@@ -223,6 +228,14 @@ struct Cfg {
   static constexpr int kPolyEvery = kFp8_ ? 4 : 8;
 };
 
+// Dynamic shared memory of fa_fwd_kernel<C, kVarlen>: the tiles and barriers
+// of C and, for variable-length batches, the first-unit table of up to
+// kMaxVarlenSeqs sequences with the per-warp totals of its scan.
+template <class C, bool kVarlen>
+constexpr int fwd_smem_bytes() {
+  return C::kSmemBytes + (kVarlen ? 4 * (kMaxVarlenSeqs + 1 + kThreads / 32) : 0);
+}
+
 // 2^x on the FMA pipe for two lanes (relieves the MUFU exp2 unit, which at
 // head dim 128 would otherwise run exactly as fast as the tensor cores eat
 // scores).  Cody-Waite range reduction x = n + f, n = round(x) via the
@@ -311,6 +324,96 @@ __device__ __forceinline__ void decode_item(const KernelParams& p, int w, int& b
   } else {  // all pairs of one head together: that head's K/V stays in L2
     bh = w / p.npairs;
     pair = w % p.npairs;
+  }
+}
+
+// Query rows of sequence b of a variable-length batch, from the offsets
+// clamped as in seq_of.
+__device__ __forceinline__ int varlen_rows(const KernelParams& p, int b) {
+  const int qa = min(max(__ldg(p.cu_q + b), 0), p.total_q);
+  const int qb = min(max(__ldg(p.cu_q + b + 1), qa), p.total_q);
+  return qb - qa;
+}
+
+// Work units of sequence b: one per pair of query tiles, for each head.
+__device__ __forceinline__ int varlen_units(const KernelParams& p, int b) {
+  const int nqt = (varlen_rows(p, b) + kBM - 1) / kBM;
+  return p.heads * ((nqt + 1) >> 1);
+}
+
+// Variable-length batches deal only the units that exist: start[b] is the
+// first unit of sequence b and start[nseq] their number, so sequences shorter
+// than the longest leave no empty units behind (CTAs that skipped through
+// empty units ran ahead of the others, and the K/V in use at once outgrew
+// L2).  Whole block, ends with __syncthreads; start holds nseq + 1 entries
+// followed by kThreads / 32 of scratch.
+__device__ inline void build_unit_table(const KernelParams& p, int* start) {
+  const int n = p.nseq;
+  const int per = (n + kThreads - 1) / kThreads;
+  const int b0 = min(n, (int)threadIdx.x * per), b1 = min(n, b0 + per);
+  int sum = 0;
+  for (int b = b0; b < b1; ++b) sum += varlen_units(p, b);
+  // Exclusive scan of the per-thread sums: within each warp, then across.
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  int* warp_total = start + n + 1;
+  if (lane == 31) warp_total[wid] = incl;
+  __syncthreads();
+  int run = incl - sum;
+  for (int i = 0; i < wid; ++i) run += warp_total[i];
+  for (int b = b0; b < b1; ++b) {
+    start[b] = run;
+    run += varlen_units(p, b);
+  }
+  if (threadIdx.x == kThreads - 1) start[n] = run;  // the last thread's run is the total
+  __syncthreads();
+}
+
+// Unit w (< start[nseq]) of a variable-length batch.  The units of one
+// sequence are consecutive; under the causal rule they run longest first with
+// the heads interleaved in groups whose K/V fit in L2 together (group_keys
+// keys per head), otherwise head by head.
+__device__ __forceinline__ void decode_varlen(const KernelParams& p, const int* start, int w, int& bh,
+                                              int& pair) {
+  int lo = 0, hi = p.nseq - 1;  // the last sequence whose first unit is <= w
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= w) lo = mid;
+    else hi = mid - 1;
+  }
+  const int b = lo, r = w - start[b];
+  const int np = (start[b + 1] - start[b]) / p.heads;  // units per head
+  int h;
+  if (p.causal) {
+    const int ka = min(max(__ldg(p.cu_k + b), 0), p.total_k);
+    const int nk = min(max(__ldg(p.cu_k + b + 1), ka), p.total_k) - ka;
+    const int gs = nk > 0 ? min(p.heads, max(1, p.group_keys / nk)) : p.heads;
+    const int g = r / (gs * np);
+    const int rr = r - g * gs * np;
+    const int gsz = min(gs, p.heads - g * gs);
+    pair = np - 1 - rr / gsz;
+    h = g * gs + rr % gsz;
+  } else {
+    h = r / np;
+    pair = r - h * np;
+  }
+  bh = b * p.heads + h;
+}
+
+// Unit w of this launch: (b * H + h, pair of query tiles, key slice).
+template <bool kVarlen>
+__device__ __forceinline__ void decode_unit(const KernelParams& p, const int* start, int w, int& bh, int& pair,
+                                            int& split) {
+  if constexpr (kVarlen) {
+    decode_varlen(p, start, w, bh, pair);
+    split = 0;
+  } else {
+    decode_item(p, w, bh, pair, split);
   }
 }
 
@@ -575,19 +678,24 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
   // Everything above is this CTA's prologue; global memory is touched only
   // after the previous grid on the stream has finished (launch overlap).
   ptx::grid_dependency_wait();
+  int* unit_start = reinterpret_cast<int*>(base_ptr + C::kOffMisc + 16);
+  int items = p.items;
+  if constexpr (kVarlen) {
+    build_unit_table(p, unit_start);
+    items = unit_start[p.nseq];
+  }
 
   if (warp == kLoadWarp) {
     // ------------------------------------------------------ TMA producer ---
     uint32_t it = 0;       // K/V ring loads issued
     uint32_t nq = 0;       // Q loads issued
     bool ok = true;
-    for (int k = 0, w = unit_of_round<!kVarlen>(0); w < p.items && ok && !p.starve_producer;
+    for (int k = 0, w = unit_of_round<!kVarlen>(0); w < items && ok && !p.starve_producer;
          w = unit_of_round<!kVarlen>(++k)) {
       int bh, pair, split;
-      decode_item(p, w, bh, pair, split);
+      decode_unit<kVarlen>(p, unit_start, w, bh, pair, split);
       const auto sq = seq_of<kVarlen>(p, bh);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
-      if (kVarlen && qt0 >= sq.nqt()) continue;  // past this sequence's end
       const int nvalid = (qt1 < sq.nqt()) ? 2 : 1;
       const int jb = split * p.kt_per_split, je = min(sq.nkt(), jb + p.kt_per_split);
       ok = wait_warp(bQEmpty, (nq & 1u) ^ 1u, abort_flag, p);
@@ -641,12 +749,11 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     int64_t v_ready = -1;         // ring index of the newest V whose load was awaited
     bool ok = true;
     const MmaCtx<C> ctx{tmem, sQ, sRing, abort_flag};
-    for (int k = 0, w = unit_of_round<!kVarlen>(0); w < p.items && ok; w = unit_of_round<!kVarlen>(++k)) {
+    for (int k = 0, w = unit_of_round<!kVarlen>(0); w < items && ok; w = unit_of_round<!kVarlen>(++k)) {
       int bh, pair, split;
-      decode_item(p, w, bh, pair, split);
+      decode_unit<kVarlen>(p, unit_start, w, bh, pair, split);
       const auto sq = seq_of<kVarlen>(p, bh);
       const int qt0 = 2 * pair, qt1 = qt0 + 1;
-      if (kVarlen && qt0 >= sq.nqt()) continue;
       const bool valid1 = qt1 < sq.nqt();
       const int jb = split * p.kt_per_split, je = min(sq.nkt(), jb + p.kt_per_split);
       slot0.begin_unit(true);
@@ -726,9 +833,9 @@ __global__ void __launch_bounds__(kThreads, 1) fa_fwd_kernel(const __grid_consta
     const float sl = p.scale_log2;
     uint32_t swait = 0, owait = 0;
     bool ok = true;
-    for (int k = 0, w = unit_of_round<!kVarlen>(0); w < p.items && ok; w = unit_of_round<!kVarlen>(++k)) {
+    for (int k = 0, w = unit_of_round<!kVarlen>(0); w < items && ok; w = unit_of_round<!kVarlen>(++k)) {
       int bh, pair, split;
-      decode_item(p, w, bh, pair, split);
+      decode_unit<kVarlen>(p, unit_start, w, bh, pair, split);
       const auto sq = seq_of<kVarlen>(p, bh);
       const int qt = 2 * pair + q;
       const int jb = split * p.kt_per_split, je = min(sq.nkt(), jb + p.kt_per_split);

@@ -225,8 +225,10 @@ FA_API int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, floa
  * q, o: bf16 [total_q, H, d]; k, v: bf16 [total_k, H, d] (token-major, d
  * fastest); lse: fp32 [H, total_q].  cu_seqlens_q / cu_seqlens_k: int32
  * device arrays of B+1 non-decreasing offsets starting at 0 and ending at
- * total_q / total_k.  max_seqlen_q must be >= every query length: rows past
- * it are not computed.  Offsets outside [0, total] are clamped on the device
+ * total_q / total_k.  max_seqlen_q, the longest query length, sizes the
+ * launch only: the work of each sequence follows its own offsets, read on
+ * the device.  Batches of more than 4096 sequences take one launch per 4096
+ * on cuda_stream.  Offsets outside [0, total] are clamped on the device
  * (so no access leaves the buffers), but such a batch has no defined result.
  * No block mask.  All pointers device memory owned by the caller, 16-byte
  * aligned (lse, cu_seqlens: 4).  Asynchronous on cuda_stream.

@@ -85,6 +85,37 @@ def test_varlen_workload_full_size():
         assert_lse_close(lse[h:h + 1], lse_ref, TOL_LSE)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_more_sequences_than_one_launch(causal):
+    # 4396 short sequences (0 to 300 tokens, empty ones among them): more
+    # than the 4096 one launch deals, so the call takes two launches, the
+    # second starting 4096 entries into the offsets.
+    g = torch.Generator().manual_seed(31)
+    lq = torch.randint(0, 301, (4396,), generator=g)
+    lq[::97] = 0
+    lq = lq.tolist()
+    _check(lq, lq, 64, causal, seed=33, H=1)
+
+
+def test_varlen_heads_split_into_l2_groups():
+    # A causal sequence long enough that the K/V of all 16 heads exceed the
+    # L2 share of one head group (15 heads of 6200 keys fit, the 16th starts a
+    # group of one), next to short and empty sequences.
+    _check([6200, 150, 0, 700], [6200, 150, 0, 700], 128, True, seed=35, H=16)
+
+
+def test_varlen_understated_max_length():
+    # max_seqlen_q only sizes the launch: a bound below the real lengths still
+    # gives every row of every sequence.
+    lq = [300, 1000, 1]
+    q, k, v, cu_q, cu_k = make_varlen(lq, lq, 2, 64, 37)
+    o, lse = _run(q, k, v, cu_q, cu_k, True, max_q=130)
+    o_ref, lse_ref = oracle.attention_varlen_ref(to_np64(q), to_np64(k), to_np64(v), cu_q.tolist(),
+                                                 cu_k.tolist(), 0.125, causal=True)
+    assert np.max(np.abs(o - o_ref)) <= TOL_O
+    assert_lse_close(lse, lse_ref, TOL_LSE)
+
+
 def test_varlen_argument_errors():
     q = torch.zeros((8, 2, 64), dtype=torch.bfloat16, device=DEV)
     cu = torch.tensor([0, 8], dtype=torch.int32, device=DEV)
