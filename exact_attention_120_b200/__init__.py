@@ -37,7 +37,7 @@ __all__ = [
     "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_bytes", "fa_fwd_splitkv_heuristic",
     "attention_forward_splitkv", "fa_bwd", "fa_bwd_workspace_bytes", "attention_backward",
     "fa_device_status", "fa_fwd_varlen", "attention_forward_varlen", "fa_fwd_fp8",
-    "attention_forward_fp8",
+    "attention_forward_fp8", "fa_fwd_host", "attention_forward_host",
     "fa_status_string", "fa_launches_per_call", "attention_forward", "FA_OK",
     "FA_ERR_INVALID_ARGUMENT", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_DEVICE_TIMEOUT",
     "MASK_BLOCK",
@@ -60,6 +60,8 @@ _SIGNATURES = {
     "fa_fwd_stream": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
                       + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                               ctypes.c_void_p]),
+    "fa_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 10 + [ctypes.c_int] * 4
+                    + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "fa_fwd_qk": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_void_p, ctypes.c_void_p]
                   + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                           ctypes.c_void_p]),
@@ -166,6 +168,13 @@ def fa_launches_per_call() -> int:
     return load_library().fa_launches_per_call()
 
 
+def fa_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, N,
+                d, scale, causal, block_mask, stream) -> int:
+    """C ``fa_fwd_host`` on raw host and device addresses and a cudaStream_t."""
+    return load_library().fa_fwd_host(q_host, k_host, v_host, o_host, lse_host, q_dev, k_dev, v_dev,
+                                      o_dev, lse_dev, B, H, N, d, scale, causal, block_mask, stream)
+
+
 def _check(t, name, dtype, shape, device=None):
     """Raise ValueError unless `t` is a contiguous CUDA tensor of `dtype` and
     `shape` (on `device` when given)."""
@@ -236,6 +245,66 @@ def attention_forward(q, k, v, causal=False, block_mask=None, scale=None, out=No
                            B, H, Nq, Nk, d, float(scale), int(bool(causal)), mask_ptr, stream)
     if st != FA_OK:
         raise FaError(st, "fa_fwd")
+    return out, lse
+
+
+def attention_forward_host(q, k, v, causal=False, block_mask=None, scale=None, out=None, lse=None,
+                           device_buffers=None, stream=None, synchronize=True):
+    """O, lse of host-resident inputs through ``fa_fwd_host``: the copies to and
+    from the device overlap the computation, chunk by chunk of heads.
+
+    q, k, v: CPU bfloat16 [B, H, N, d], contiguous (page-locked for the copies
+    to overlap).  out / lse: CPU bf16 [B, H, N, d] / fp32 [B, H, N] to write
+    (page-locked ones are allocated when None).  device_buffers: None or the
+    CUDA tensors (q, k, v, o, lse) the data pass through (allocated on the
+    current device when None).  block_mask: None or a CUDA uint8 tensor as for
+    attention_forward.  With ``synchronize`` the device is synchronised before
+    returning, so out and lse are ready; otherwise they are complete once the
+    stream has passed this call, and q, k, v, out and lse must stay alive until
+    then (the copies are not known to torch's pinned-memory cache, which would
+    otherwise hand their memory to the next pinned tensor).  Returns (out, lse).
+    """
+    import torch
+
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    B, H, N, d = q.shape
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H, N, d):
+            raise ValueError(f"{name} must be a contiguous CPU bfloat16 tensor of shape {(B, H, N, d)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    for t, name, dt, shape in ((out, "out", torch.bfloat16, (B, H, N, d)),
+                               (lse, "lse", torch.float32, (B, H, N))):
+        if t.dtype != dt or t.is_cuda or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be a contiguous CPU {dt} tensor of shape {shape}")
+    dev = torch.device("cuda", torch.cuda.current_device()) if block_mask is None else block_mask.device
+    if device_buffers is None:
+        device_buffers = (torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                          torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                          torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                          torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev),
+                          torch.empty((B, H, N), dtype=torch.float32, device=dev))
+    qd, kd, vd, od, ld = device_buffers
+    dev = qd.device
+    for t, name in ((qd, "q_dev"), (kd, "k_dev"), (vd, "v_dev"), (od, "o_dev")):
+        _check(t, name, torch.bfloat16, (B, H, N, d), dev)
+    _check(ld, "lse_dev", torch.float32, (B, H, N), dev)
+    mask_ptr = _check_mask(block_mask, B, H, N, N, dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        st = fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), ld.data_ptr(),
+                         B, H, N, d, float(scale), int(bool(causal)), mask_ptr, stream)
+        if st != FA_OK:
+            raise FaError(st, "fa_fwd_host")
+        if synchronize:
+            torch.cuda.synchronize(dev)
     return out, lse
 
 

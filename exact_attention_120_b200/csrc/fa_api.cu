@@ -39,6 +39,7 @@ thread_local int t_last_cuda_error = 0;
 
 constexpr unsigned long long kWaitTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s per wait
 constexpr int kMaxDevices = 64;
+constexpr int kHostChunks = 8;  // fa_fwd_host: chunks of heads in flight
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -51,6 +52,15 @@ struct DeviceState {
   int num_sms = 0;
   int* status_word = nullptr;     // device address of g_fa_status
   void* noalloc_scratch = nullptr;  // device address of g_noalloc_scratch
+  // fa_fwd_host: one copy stream per direction and the events that order the
+  // chunks, created on its first call on the device.  The mutex keeps the
+  // enqueue of one call whole when several host threads call at once.
+  std::once_flag host_once;
+  int host_status = FA_ERR_CUDA;
+  std::mutex host_mu;
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in_done = nullptr, ev_done = nullptr;
+  cudaEvent_t ev_in[kHostChunks] = {}, ev_comp[kHostChunks] = {};
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -118,6 +128,19 @@ int get_device_state(DeviceState** out) {
   if (st.status != FA_OK) return st.status;
   *out = &st;
   return FA_OK;
+}
+
+int setup_host_streams(DeviceState& st) {
+  cudaError_t e = cudaStreamCreateWithFlags(&st.copy_in, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&st.copy_out, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st.ev_start, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st.ev_in_done, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st.ev_done, cudaEventDisableTiming);
+  for (int c = 0; c < kHostChunks && e == cudaSuccess; ++c) {
+    e = cudaEventCreateWithFlags(&st.ev_in[c], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&st.ev_comp[c], cudaEventDisableTiming);
+  }
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
 int get_encoder() {
@@ -312,7 +335,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                int Nq, int Nk, int d, float scale, int causal, const uint8_t* block_mask,
                void* cuda_stream, unsigned long long timeout_ns, int starve_producer,
                const FwdGeom& g, DeviceState* st, void* workspace = nullptr, bool fp8 = false,
-               float q_descale = 1.f, float k_descale = 1.f, float v_descale = 1.f) {
+               float q_descale = 1.f, float k_descale = 1.f, float v_descale = 1.f,
+               bool allow_overlap = true) {
   const long long bh = g.bh, nqt = g.nqt, nkt = g.nkt, npairs = g.npairs;
   const int splits = g.splits, kt_per_split = g.kt_per_split;
   const size_t rows = g.rows;
@@ -360,7 +384,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   // ---- launch: persistent grid, one CTA per SM
   const int grid = p.items < st->num_sms ? p.items : st->num_sms;
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
-  const bool overlap = p.items <= 2 * st->num_sms;  // short grids: launch overlap pays
+  const bool overlap = allow_overlap && p.items <= 2 * st->num_sms;  // short grids: launch overlap pays
   cudaError_t e;
   if (fp8)
     e = launch(overlap, fa::fa_fwd_kernel<fa::Cfg<128, true>>, grid, fa::kThreads, fa::Cfg<128, true>::kSmemBytes, stream, p);
@@ -669,6 +693,89 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
            int d, float scale, int causal, const uint8_t* block_mask) {
   return fa_fwd_stream(q, k, v, o, lse, B, H, N, d, scale, causal, block_mask, nullptr);
+}
+
+int fa_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
+                int B, int H, int N, int d, float scale, int causal, const uint8_t* block_mask,
+                void* cuda_stream) {
+  // Host checks first, with no CUDA call.
+  if (!q_host || !k_host || !v_host || !o_host || !lse_host) return FA_ERR_INVALID_ARGUMENT;
+  FwdGeom g;
+  int rc = check_fwd_args(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, N, N, d, scale, causal,
+                          block_mask, 1, false, 1.f, 1.f, 1.f, g);
+  if (rc != FA_OK) return rc;
+  const size_t head_bytes = (size_t)N * d * 2;  // one head of Q, K, V or O
+  const size_t qkv_bytes = (size_t)g.bh * head_bytes;
+  if (outputs_alias({{o_host, qkv_bytes}, {lse_host, g.rows * sizeof(float)}},
+                    {{q_host, qkv_bytes}, {k_host, qkv_bytes}, {v_host, qkv_bytes}}))
+    return FA_ERR_INVALID_ARGUMENT;
+
+  DeviceState* st = nullptr;
+  if ((rc = get_device_state(&st)) != FA_OK) return rc;
+  for (const void* ptr : std::initializer_list<const void*>{q_dev, k_dev, v_dev, o_dev, lse_dev})
+    if (!is_device_pointer(ptr)) return FA_ERR_INVALID_ARGUMENT;
+  if (block_mask && !is_device_pointer(block_mask)) return FA_ERR_INVALID_ARGUMENT;
+  for (const void* ptr : std::initializer_list<const void*>{q_host, k_host, v_host, o_host, lse_host})
+    if (is_device_pointer(ptr)) return FA_ERR_INVALID_ARGUMENT;
+  std::call_once(st->host_once, [&] { st->host_status = setup_host_streams(*st); });
+  if (st->host_status != FA_OK) return st->host_status;
+  std::lock_guard<std::mutex> lock(st->host_mu);
+
+  // Chunk c of whole heads [h0, h0 + hn): copy in on copy_in, compute on the
+  // caller's stream once its copy has landed, copy out on copy_out once it is
+  // computed.  Each chunk is a batch of hn heads for the kernel.
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  const long long nchunks = std::min<long long>(kHostChunks, g.bh);
+  const long long per = (g.bh + nchunks - 1) / nchunks;
+  const size_t mask_head = (size_t)g.nqt * g.nkt;
+  cudaError_t e = cudaEventRecord(st->ev_start, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st->copy_in, st->ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st->copy_out, st->ev_start, 0);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int c = 0;
+  for (long long h0 = 0; h0 < g.bh && e == cudaSuccess && rc == FA_OK; h0 += per, ++c) {
+    const int hn = (int)std::min(per, g.bh - h0);
+    const size_t off = (size_t)h0 * head_bytes, bytes = (size_t)hn * head_bytes;
+    const size_t loff = (size_t)h0 * N * sizeof(float), lbytes = (size_t)hn * N * sizeof(float);
+    char* qd = static_cast<char*>(q_dev) + off;
+    char* kd = static_cast<char*>(k_dev) + off;
+    char* vd = static_cast<char*>(v_dev) + off;
+    char* od = static_cast<char*>(o_dev) + off;
+    float* ld = reinterpret_cast<float*>(reinterpret_cast<char*>(lse_dev) + loff);
+    e = cudaMemcpyAsync(qd, static_cast<const char*>(q_host) + off, bytes, cudaMemcpyHostToDevice, st->copy_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(kd, static_cast<const char*>(k_host) + off, bytes, cudaMemcpyHostToDevice, st->copy_in);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(vd, static_cast<const char*>(v_host) + off, bytes, cudaMemcpyHostToDevice, st->copy_in);
+    if (e == cudaSuccess) e = cudaEventRecord(st->ev_in[c], st->copy_in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, st->ev_in[c], 0);
+    if (e != cudaSuccess) break;
+    FwdGeom gc;
+    const uint8_t* mc = block_mask ? block_mask + (size_t)h0 * mask_head : nullptr;
+    rc = check_fwd_args(qd, kd, vd, od, ld, 1, hn, N, N, d, scale, causal, mc, 1, false, 1.f, 1.f, 1.f, gc);
+    if (rc == FA_OK)
+      rc = launch_fwd(qd, kd, vd, od, ld, 1, hn, N, N, d, scale, causal, mc, s, kWaitTimeoutNs, 0, gc, st,
+                      nullptr, false, 1.f, 1.f, 1.f, /*allow_overlap=*/false);
+    if (rc != FA_OK) break;
+    e = cudaEventRecord(st->ev_comp[c], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st->copy_out, st->ev_comp[c], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<char*>(o_host) + off, od, bytes, cudaMemcpyDeviceToHost, st->copy_out);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(reinterpret_cast<char*>(lse_host) + loff, ld, lbytes, cudaMemcpyDeviceToHost,
+                          st->copy_out);
+  }
+  // Whatever was enqueued, the caller's stream waits for both copy streams,
+  // so that no copy of this call outlives it unordered.
+  cudaError_t e2 = cudaEventRecord(st->ev_done, st->copy_out);
+  if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(s, st->ev_done, 0);
+  if (e2 == cudaSuccess) e2 = cudaEventRecord(st->ev_in_done, st->copy_in);
+  if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(s, st->ev_in_done, 0);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (rc != FA_OK) return rc;
+  if (e2 != cudaSuccess) return cuda_fail(e2);
+  return FA_OK;
 }
 
 int fa_device_status(void* cuda_stream) {

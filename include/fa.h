@@ -95,6 +95,41 @@ FA_API int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, f
                   void* cuda_stream);
 
 /*
+ * The forward pass of fa_fwd_stream for inputs and outputs in host memory,
+ * with the host<->device transfers overlapped with the computation.
+ *
+ * q_host, k_host, v_host (bf16 [B,H,N,d]), o_host (bf16 [B,H,N,d]) and
+ * lse_host (fp32 [B,H,N]) are host memory owned by the caller; page-locked
+ * memory lets the copies overlap each other and the kernels (pageable memory
+ * works, but its copies do not overlap).  q_dev ... lse_dev are device
+ * buffers of the same sizes, owned by the caller, through which the data
+ * pass (afterwards they hold the inputs and the results as well).
+ * block_mask: NULL or device memory, as for fa_fwd.
+ *
+ * The B*H heads are taken in up to 8 chunks of whole heads.  Chunk c's Q, K
+ * and V are copied in on an internal stream while the chunks before it are
+ * computed on cuda_stream and their O and lse are copied out on a second
+ * internal stream (a copy engine per direction).  Each chunk is computed by
+ * the same kernel as fa_fwd_stream, so the results are bit for bit those of
+ * fa_fwd_stream.  Ordering: the call's work starts after the work enqueued on
+ * cuda_stream before it, and everything it does, the copies into o_host and
+ * lse_host included, is complete once cuda_stream has passed the point of
+ * the call's return: synchronise cuda_stream before reading o_host.  The
+ * host buffers must stay valid until then.  The internal streams and events
+ * are created on the first call on each device and kept.
+ *
+ * Returns FA_OK, FA_ERR_INVALID_ARGUMENT (a null pointer, a *_dev pointer
+ * that is not device memory or a *_host pointer that is, sizes, scale or
+ * causal as for fa_fwd, o_dev / lse_dev overlapping an input buffer, o_host /
+ * lse_host overlapping q_host, k_host, v_host or each other),
+ * FA_ERR_UNSUPPORTED or FA_ERR_CUDA.
+ */
+FA_API int fa_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                       float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                       float* lse_dev, int B, int H, int N, int d, float scale, int causal,
+                       const uint8_t* block_mask, void* cuda_stream);
+
+/*
  * Attention with Nq query rows and Nk keys per (b, h) -- cross-attention, or
  * decoding against a key/value cache.  q, o: [B, H, Nq, d]; k, v: [B, H, Nk, d];
  * lse: [B, H, Nq]; block_mask: NULL or [B, H, ceil(Nq/128), ceil(Nk/128)].
@@ -283,10 +318,10 @@ FA_API const char* fa_status_string(int status);
 /* The cudaError_t value behind the last FA_ERR_CUDA on this host thread. */
 FA_API int fa_last_cuda_error(void);
 
-/* Number of kernel launches one fa_fwd / fa_fwd_qk / fa_fwd_varlen /
- * fa_fwd_fp8 call makes (constant: 1).  fa_fwd_splitkv with more than one
- * slice makes 2 (the forward and the merge), fa_bwd makes 2 (the dQ and the
- * dK/dV launches). */
+/* Number of kernel launches one fa_fwd / fa_fwd_qk / fa_fwd_fp8 call makes
+ * (constant: 1).  fa_fwd_varlen makes one per 4096 sequences, fa_fwd_host one
+ * per chunk of heads, fa_fwd_splitkv with more than one slice 2 (the forward
+ * and the merge), fa_bwd 2 (the dQ and the dK/dV launches). */
 FA_API int fa_launches_per_call(void);
 
 #ifdef __cplusplus

@@ -106,6 +106,36 @@ def test_noalloc_argument_errors_before_any_cuda_call(lib):
     assert call(B=1, H=1, Nq=16257, Nk=256, splits=2) == fa.FA_ERR_UNSUPPORTED
 
 
+def test_host_entry_argument_errors_before_any_cuda_call(lib):
+    """fa_fwd_host checks pointers, sizes and overlaps before any CUDA call."""
+    p = 1 << 24  # never dereferenced: every case fails validation first
+    names = ["qh", "kh", "vh", "oh", "lh", "qd", "kd", "vd", "od", "ld", "B", "H", "N", "d", "scale",
+             "causal", "mask", "stream"]
+    # host buffers at 11p.., device buffers at p..; each tensor is 16 KB
+    # (one head, N = 128, d = 64), lse 512 B
+    base = [p * 11, p * 12, p * 13, p * 14, p * 15, p, p * 2, p * 3, p * 4, p * 5, 1, 1, 128, 64, 0.125,
+            0, None, None]
+
+    def call(**kw):
+        a = list(base)
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return lib.fa_fwd_host(*a)
+
+    for name in ("qh", "kh", "vh", "oh", "lh", "qd", "kd", "vd", "od", "ld"):
+        assert call(**{name: None}) == fa.FA_ERR_INVALID_ARGUMENT, name
+    assert call(B=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(N=0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(scale=-1.0) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(causal=2) == fa.FA_ERR_INVALID_ARGUMENT
+    assert call(d=32) == fa.FA_ERR_UNSUPPORTED
+    assert call(qd=p + 8) == fa.FA_ERR_INVALID_ARGUMENT          # device q misaligned
+    assert call(od=p * 2 + 4096) == fa.FA_ERR_INVALID_ARGUMENT   # device o inside device k
+    assert call(oh=p * 13 + 4096) == fa.FA_ERR_INVALID_ARGUMENT  # host o inside host v
+    assert call(lh=p * 11 + 64) == fa.FA_ERR_INVALID_ARGUMENT    # host lse inside host q
+    assert call(lh=p * 14 + 16384 - 4) == fa.FA_ERR_INVALID_ARGUMENT  # host lse on host o's end
+
+
 def test_splitkv_workspace_size(lib):
     # [splits][rows][d] fp32 partial outputs + [splits][rows] fp32 lse
     assert fa.fa_fwd_splitkv_workspace_bytes(2, 4, 1, 16384, 128, 8) == 8 * 8 * 129 * 4
