@@ -729,7 +729,8 @@ def run_ours(args, info):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "entry": job.e2e_entry},
         "ms_per_step_percentiles": {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9),
-                                    "steps": len(per_ms)},
+                                    "steps": len(per_ms),
+                                    "taken": "after the timed region, one event pair per launch"},
         "host_us_per_call": statistics.median(host_us),
         "gpu_launches": args.steps * job.launches_per_step,
         "clocks": clocks,
