@@ -39,7 +39,9 @@ thread_local int t_last_cuda_error = 0;
 
 constexpr unsigned long long kWaitTimeoutNs = 1000ull * 1000ull * 1000ull;  // 1 s per wait
 constexpr int kMaxDevices = 64;
-constexpr int kHostChunks = 8;  // fa_fwd_host: chunks of heads in flight
+// fa_fwd_host: chunks of heads.  Measured on B=1, H=16, N=16384, d=128 from
+// pinned memory: 4, 8, 16 chunks -> 4.73, 4.58, 4.54 ms per call.
+constexpr int kHostChunks = 16;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

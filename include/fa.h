@@ -106,7 +106,7 @@ FA_API int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, f
  * pass (afterwards they hold the inputs and the results as well).
  * block_mask: NULL or device memory, as for fa_fwd.
  *
- * The B*H heads are taken in up to 8 chunks of whole heads.  Chunk c's Q, K
+ * The B*H heads are taken in up to 16 chunks of whole heads.  Chunk c's Q, K
  * and V are copied in on an internal stream while the chunks before it are
  * computed on cuda_stream and their O and lse are copied out on a second
  * internal stream (a copy engine per direction).  Each chunk is computed by
