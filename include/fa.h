@@ -116,7 +116,8 @@ FA_API int fa_fwd_stream(const void* q, const void* k, const void* v, void* o, f
  * lse_host included, is complete once cuda_stream has passed the point of
  * the call's return: synchronise cuda_stream before reading o_host.  The
  * host buffers must stay valid until then.  The internal streams and events
- * are created on the first call on each device and kept.
+ * are created on the first call on each device and kept; calls on one device
+ * share them, so the copies of concurrent calls run one call after another.
  *
  * Returns FA_OK, FA_ERR_INVALID_ARGUMENT (a null pointer, a *_dev pointer
  * that is not device memory or a *_host pointer that is, sizes, scale or
