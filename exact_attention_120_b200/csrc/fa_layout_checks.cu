@@ -31,6 +31,8 @@ constexpr bool fwd_layout_ok() {
     static_assert(kPCols <= 128, "P wider than S");
   }
   static_assert(C::kSmemBytes <= kMaxSmemPerCta, "shared memory over the per-CTA limit");
+  // Variable-length batches add the table of the sequences' first work units.
+  static_assert(fwd_smem_bytes<C, true>() <= kMaxSmemPerCta, "variable-length table over the per-CTA limit");
   static_assert(C::kOffRing % 1024 == 0 && C::kTileBytes % 1024 == 0, "swizzle-atom alignment");
   static_assert(C::kBoxes * C::kBoxBytes == C::kTileBytes, "tile = whole TMA boxes");
   static_assert(C::kOffBar % 8 == 0, "mbarrier alignment");
