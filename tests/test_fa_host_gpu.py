@@ -106,3 +106,41 @@ def test_host_entry_rejects_swapped_memory_kinds():
     # a device pointer where host memory belongs, and the reverse
     assert lib.fa_fwd_host(qd.data_ptr(), *args[1:], *dargs, *tail) == fa.FA_ERR_INVALID_ARGUMENT
     assert lib.fa_fwd_host(*args, qh.data_ptr(), *dargs[1:], *tail) == fa.FA_ERR_INVALID_ARGUMENT
+
+
+def test_host_entry_from_two_threads_on_two_streams():
+    # Two host threads call at once, each with its own buffers and stream: the
+    # calls share the library's copy streams (one call's enqueue is kept whole)
+    # and each must return its own results.
+    import threading
+
+    B, H, N, d = 1, 6, 1024, 64
+    jobs = []
+    for seed in (51, 52):
+        q, k, v = make_qkv(B, H, N, d, seed=seed)
+        bufs = tuple(torch.empty((B, H, N, d), dtype=torch.bfloat16, device=DEV) for _ in range(4)) + (
+            torch.empty((B, H, N), dtype=torch.float32, device=DEV),)
+        out = (_pinned(torch.empty((B, H, N, d), dtype=torch.bfloat16)),
+               _pinned(torch.empty((B, H, N), dtype=torch.float32)))
+        jobs.append(dict(qkv=(q, k, v), host=[_pinned(t) for t in (q, k, v)], bufs=bufs,
+                         stream=torch.cuda.Stream(DEV), out=out))
+
+    def run(job):
+        with torch.cuda.device(DEV):
+            for _ in range(3):
+                fa.attention_forward_host(*job["host"], out=job["out"][0], lse=job["out"][1],
+                                          device_buffers=job["bufs"], stream=job["stream"].cuda_stream,
+                                          synchronize=False)
+            job["stream"].synchronize()
+
+    threads = [threading.Thread(target=run, args=(j,)) for j in jobs]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    torch.cuda.synchronize()
+    for job in jobs:
+        q, k, v = job["qkv"]
+        o_ref, l_ref = fa.attention_forward(q.to(DEV), k.to(DEV), v.to(DEV))
+        o, l_ = job["out"]
+        assert torch.equal(o, o_ref.cpu()) and torch.equal(l_, l_ref.cpu())
