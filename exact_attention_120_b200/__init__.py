@@ -258,8 +258,9 @@ def attention_forward_host(q, k, v, causal=False, block_mask=None, scale=None, o
     (page-locked ones are allocated when None).  device_buffers: None or the
     CUDA tensors (q, k, v, o, lse) the data pass through (allocated on the
     current device when None).  block_mask: None or a CUDA uint8 tensor as for
-    attention_forward.  With ``synchronize`` the device is synchronised before
-    returning, so out and lse are ready; otherwise they are complete once the
+    attention_forward.  With ``synchronize`` the call's stream (the device, for
+    a raw stream handle) is synchronised before returning, so out and lse are
+    ready; otherwise they are complete once the
     stream has passed this call, and q, k, v, out and lse must stay alive until
     then (the copies are not known to torch's pinned-memory cache, which would
     otherwise hand their memory to the next pinned tensor).  Returns (out, lse).
@@ -295,8 +296,9 @@ def attention_forward_host(q, k, v, causal=False, block_mask=None, scale=None, o
         _check(t, name, torch.bfloat16, (B, H, N, d), dev)
     _check(ld, "lse_dev", torch.float32, (B, H, N), dev)
     mask_ptr = _check_mask(block_mask, B, H, N, N, dev)
+    torch_stream = torch.cuda.current_stream(dev) if stream is None else None
     if stream is None:
-        stream = torch.cuda.current_stream(dev).cuda_stream
+        stream = torch_stream.cuda_stream
     with torch.cuda.device(dev):
         st = fa_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                          qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), ld.data_ptr(),
@@ -304,7 +306,12 @@ def attention_forward_host(q, k, v, causal=False, block_mask=None, scale=None, o
         if st != FA_OK:
             raise FaError(st, "fa_fwd_host")
         if synchronize:
-            torch.cuda.synchronize(dev)
+            # The call's work ends on its stream: wait for that stream (for a raw
+            # handle passed in, for the device).
+            if torch_stream is not None:
+                torch_stream.synchronize()
+            else:
+                torch.cuda.synchronize(dev)
     return out, lse
 
 
