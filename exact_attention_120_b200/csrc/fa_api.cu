@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/fa.h: argument validation,
-// TMA descriptor encoding, per-device set-up and the kernel launch.
+// TMA descriptor encoding, per-device set-up, the kernel launches, and the
+// chunked copy pipeline of the host-buffer forward (fa_fwd_host).
 //
 // Nothing here computes any part of attention: every step runs in the
 // kernels (fa_fwd_kernel and its instantiations, fa_combine_kernel for split
